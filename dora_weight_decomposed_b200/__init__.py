@@ -1,0 +1,233 @@
+"""DoRA adapter layer for B200 (sm_100a): Python binding of libdora_b200.so.
+
+The functions here only marshal arguments: they check tensor dtypes, devices
+and shapes, allocate outputs and the workspace with torch (device memory and
+streams are the only things torch provides), and call the C ABI declared in
+include/dora.h. Every step of the computation runs in the library's CUDA
+kernels; if the library is missing the import of this module still works but
+every call raises.
+
+    norm, g, gm1 = dora_norm(W0, A, B, m, s)
+    y, su, pre   = dora_forward(x, W0, A, B, gm1, s)
+    dm, dA, dB, dx = dora_backward(dy, x, W0, A, B, norm, g, su, pre, s)
+
+bf16 tensors use the tcgen05 tensor-core path; fp32 tensors use the SIMT path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+__all__ = ["DoraError", "load_library", "library_path", "dora_workspace_size", "dora_norm", "dora_forward",
+           "dora_backward", "dora_device_status", "dora_last_error", "dora_version", "DORA_OP_NORM",
+           "DORA_OP_FORWARD", "DORA_OP_BACKWARD", "STATUS_NAMES", "EXPORTED_SYMBOLS"]
+
+DORA_BF16, DORA_FP32 = 0, 1
+DORA_OP_NORM, DORA_OP_FORWARD, DORA_OP_BACKWARD = 0, 1, 2
+STATUS_NAMES = {0: "DORA_OK", 1: "DORA_EINVAL", 2: "DORA_EUNSUPPORTED", 3: "DORA_EWORKSPACE", 4: "DORA_ECUDA",
+                5: "DORA_ETIMEOUT"}
+EXPORTED_SYMBOLS = ("dora_workspace_size", "dora_norm", "dora_forward", "dora_backward", "dora_device_status",
+                    "dora_last_error", "dora_version")
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libdora_b200.so")
+
+
+class DoraError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class DoraDesc(ctypes.Structure):
+    _fields_ = [("d_out", ctypes.c_int64), ("d_in", ctypes.c_int64), ("r", ctypes.c_int64),
+                ("dtype", ctypes.c_int), ("s", ctypes.c_float)]
+
+
+_lib = None
+_lib_lock = threading.Lock()
+
+
+def load_library() -> ctypes.CDLL:
+    """Load the in-tree library (raises if it has not been built)."""
+    global _lib
+    with _lib_lock:
+        if _lib is not None:
+            return _lib
+        path = library_path()
+        if not os.path.exists(path):
+            raise ImportError(f"{path} is missing; build it with `python -m dora_weight_decomposed_b200.build`")
+        lib = ctypes.CDLL(path)
+        P, I64, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+        DP = ctypes.POINTER(DoraDesc)
+        lib.dora_workspace_size.argtypes = [DP, I64, ctypes.c_int]
+        lib.dora_workspace_size.restype = SZ
+        lib.dora_norm.argtypes = [DP, P, P, P, P, P, P, P, P, SZ, P]
+        lib.dora_norm.restype = ctypes.c_int
+        lib.dora_forward.argtypes = [DP, I64, P, P, P, P, P, P, P, P, P, SZ, P]
+        lib.dora_forward.restype = ctypes.c_int
+        lib.dora_backward.argtypes = [DP, I64, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        lib.dora_backward.restype = ctypes.c_int
+        lib.dora_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint)]
+        lib.dora_device_status.restype = ctypes.c_int
+        lib.dora_last_error.argtypes = []
+        lib.dora_last_error.restype = ctypes.c_char_p
+        lib.dora_version.argtypes = []
+        lib.dora_version.restype = ctypes.c_int
+        _lib = lib
+        return lib
+
+
+def dora_last_error() -> str:
+    return load_library().dora_last_error().decode()
+
+
+def dora_version() -> int:
+    return load_library().dora_version()
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        raise DoraError(status, dora_last_error())
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _desc(d_out: int, d_in: int, r: int, dtype, s: float) -> DoraDesc:
+    torch = _torch()
+    if dtype == torch.bfloat16:
+        code = DORA_BF16
+    elif dtype == torch.float32:
+        code = DORA_FP32
+    else:
+        raise TypeError(f"DoRA tensors must be bfloat16 or float32, got {dtype}")
+    return DoraDesc(int(d_out), int(d_in), int(r), code, float(s))
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream_ptr(stream) -> int | None:
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream or None
+
+
+def _shape(t, shape, name):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def dora_workspace_size(d_out: int, d_in: int, r: int, dtype, s: float, T: int, op: int) -> int:
+    d = _desc(d_out, d_in, r, dtype, s)
+    return int(load_library().dora_workspace_size(ctypes.byref(d), int(T), int(op)))
+
+
+def _workspace(desc: DoraDesc, T: int, op: int, device, ws):
+    torch = _torch()
+    need = int(load_library().dora_workspace_size(ctypes.byref(desc), int(T), int(op)))
+    if ws is not None:
+        return ws, ws.numel() * ws.element_size()
+    if need == 0:
+        return None, 0
+    return torch.empty(need, dtype=torch.uint8, device=device), need
+
+
+def dora_norm(W0, A, B, m, s: float, *, norm_out=None, g_out=None, gm1_out=None, ws=None, stream=None):
+    """Per-row norm C of W0 + s B A (factored form), g = m / C, gm1 = (m - C) / C."""
+    torch = _torch()
+    lib = load_library()
+    d_out, d_in = W0.shape
+    r = A.shape[0]
+    _shape(A, (r, d_in), "A")
+    _shape(B, (d_out, r), "B")
+    _shape(m, (d_out,), "m")
+    if A.dtype != W0.dtype or B.dtype != W0.dtype or m.dtype != torch.float32:
+        raise TypeError("W0, A, B share one dtype; m is float32")
+    desc = _desc(d_out, d_in, r, W0.dtype, s)
+    f32 = dict(dtype=torch.float32, device=W0.device)
+    norm_out = torch.empty(d_out, **f32) if norm_out is None else norm_out
+    g_out = torch.empty(d_out, **f32) if g_out is None else g_out
+    gm1_out = torch.empty(d_out, **f32) if gm1_out is None else gm1_out
+    wsb, nbytes = _workspace(desc, 0, DORA_OP_NORM, W0.device, ws)
+    _check(lib.dora_norm(ctypes.byref(desc), _ptr(W0), _ptr(A), _ptr(B), _ptr(m), _ptr(norm_out), _ptr(g_out),
+                         _ptr(gm1_out), _ptr(wsb), nbytes, _stream_ptr(stream)))
+    return norm_out, g_out, gm1_out
+
+
+def dora_forward(x, W0, A, B, gm1, s: float, *, save_for_backward: bool = True, y=None, su_save=None,
+                 pre_save=None, ws=None, stream=None):
+    """y = x (diag(g) (W0 + s B A))^T composed as pre + gm1 * pre.
+
+    Returns (y, su, pre); su = s x A^T and pre (the un-scaled output) are the
+    tensors dora_backward needs (None when save_for_backward is False).
+    """
+    torch = _torch()
+    lib = load_library()
+    T, d_in = x.shape
+    d_out = W0.shape[0]
+    r = A.shape[0]
+    _shape(W0, (d_out, d_in), "W0")
+    _shape(A, (r, d_in), "A")
+    _shape(B, (d_out, r), "B")
+    _shape(gm1, (d_out,), "gm1")
+    desc = _desc(d_out, d_in, r, W0.dtype, s)
+    dev = x.device
+    y = torch.empty(T, d_out, dtype=x.dtype, device=dev) if y is None else y
+    if save_for_backward:
+        su_save = torch.empty(T, r, dtype=x.dtype, device=dev) if su_save is None else su_save
+        pre_save = torch.empty(T, d_out, dtype=x.dtype, device=dev) if pre_save is None else pre_save
+    wsb, nbytes = _workspace(desc, T, DORA_OP_FORWARD, dev, ws)
+    _check(lib.dora_forward(ctypes.byref(desc), T, _ptr(x), _ptr(W0), _ptr(A), _ptr(B), _ptr(gm1), _ptr(y),
+                            _ptr(su_save), _ptr(pre_save), _ptr(wsb), nbytes, _stream_ptr(stream)))
+    return y, su_save, pre_save
+
+
+def dora_backward(dy, x, W0, A, B, norm, g, su_save, pre_save, s: float, *, need_dx: bool = True, dm=None,
+                  dA=None, dB=None, dx=None, ws=None, stream=None):
+    """Detached-norm gradients (dm, dA, dB, dx); dx is None when need_dx is False."""
+    torch = _torch()
+    lib = load_library()
+    T, d_in = x.shape
+    d_out = W0.shape[0]
+    r = A.shape[0]
+    _shape(dy, (T, d_out), "dy")
+    _shape(su_save, (T, r), "su_save")
+    _shape(pre_save, (T, d_out), "pre_save")
+    desc = _desc(d_out, d_in, r, W0.dtype, s)
+    dev = x.device
+    dm = torch.empty(d_out, dtype=torch.float32, device=dev) if dm is None else dm
+    dA = torch.empty(r, d_in, dtype=x.dtype, device=dev) if dA is None else dA
+    dB = torch.empty(d_out, r, dtype=x.dtype, device=dev) if dB is None else dB
+    if need_dx and dx is None:
+        dx = torch.empty(T, d_in, dtype=x.dtype, device=dev)
+    if not need_dx:
+        dx = None
+    wsb, nbytes = _workspace(desc, T, DORA_OP_BACKWARD, dev, ws)
+    _check(lib.dora_backward(ctypes.byref(desc), T, _ptr(dy), _ptr(x), _ptr(W0), _ptr(A), _ptr(B), _ptr(norm),
+                             _ptr(g), _ptr(su_save), _ptr(pre_save), _ptr(dm), _ptr(dA), _ptr(dB), _ptr(dx),
+                             _ptr(wsb), nbytes, _stream_ptr(stream)))
+    return dm, dA, dB, dx
+
+
+def dora_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the kernels' timeout flags."""
+    flags = ctypes.c_uint(0)
+    st = load_library().dora_device_status(_stream_ptr(stream), ctypes.byref(flags))
+    if st not in (0, 5):
+        _check(st)
+    return int(flags.value)

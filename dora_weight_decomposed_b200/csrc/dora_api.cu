@@ -1,0 +1,278 @@
+// C ABI of the DoRA layer library: argument checks, workspace planning and
+// dispatch to the bf16 (tcgen05) or fp32 (SIMT) implementation. No call
+// allocates device memory or synchronises (except dora_device_status).
+#include <cmath>
+#include <cstring>
+#include <string>
+
+#include "dora_internal.h"
+
+namespace dora {
+
+static thread_local std::string t_last_error;
+
+void set_error(const std::string& msg) { t_last_error = msg; }
+
+int device_sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+    cudaGetLastError();
+    return 148;  // no device visible: plan for a full B200
+  }
+  return sms;
+}
+
+static inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+static inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Pick how many K splits a GEMM with `tiles` output tiles and `kb` k-blocks
+// gets: minimise (waves of one-CTA-per-SM) x (k-blocks per CTA + fixed cost).
+static Split choose_split(int64_t tiles, int64_t kb, int sms) {
+  Split best;
+  best.splits = 1;
+  best.kb_per_split = (int)std::max<int64_t>(kb, 1);
+  if (kb <= 1 || tiles <= 0) return best;
+  const double fixed_cost = 4.0;
+  double best_t = 1e300;
+  for (int64_t n = 1; n <= std::min<int64_t>(kb, 64); ++n) {
+    const int64_t kps = cdiv(kb, n);
+    const int64_t ns = cdiv(kb, kps);
+    const int64_t waves = cdiv(tiles * ns, sms);
+    const double t = (double)waves * ((double)kps + fixed_cost);
+    if (t < best_t - 1e-9) {
+      best_t = t;
+      best.splits = (int)ns;
+      best.kb_per_split = (int)kps;
+    }
+  }
+  return best;
+}
+
+static int bn_skinny(int64_t r) { return r <= 16 ? 16 : r <= 32 ? 32 : r <= 64 ? 64 : 128; }
+
+Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
+  Plan p;
+  p.sms = device_sm_count();
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const int64_t r = d.r, d_in = d.d_in, d_out = d.d_out;
+  if (d.dtype == DORA_BF16) {
+    if (op == DORA_OP_NORM) {
+      const int64_t gram_tiles = cdiv(r, 128) * cdiv(r, bn_skinny(r));
+      p.gram = choose_split(gram_tiles, cdiv(d_in, 64), p.sms);
+      p.off_gram_part = take((size_t)p.gram.splits * r * r * 4);
+      p.off_gs = take((size_t)r * 2 * cdiv(r, 64) * 64 * 2);
+      p.norm = choose_split(cdiv(d_out, 128), cdiv(d_in, 64) + 2 * cdiv(r, 64), p.sms);
+      p.off_norm_part = take((size_t)p.norm.splits * d_out * 4);
+    } else if (op == DORA_OP_FORWARD && T > 0) {
+      p.u_bn = bn_skinny(r);
+      p.u = choose_split(cdiv(T, 128) * cdiv(r, p.u_bn), cdiv(d_in, 64), p.sms);
+      if (p.u.splits > 1) p.off_u_part = take((size_t)p.u.splits * T * r * 4);
+      p.off_su = take((size_t)T * r * 2);
+    } else if (op == DORA_OP_BACKWARD && T > 0) {
+      p.off_dz = take((size_t)T * d_out * 2);
+      p.dm_rowblocks = (int)cdiv(T, 256);
+      p.off_dm_part = take((size_t)p.dm_rowblocks * d_out * 4);
+      p.r_bn_mn = r <= 64 ? 64 : 128;
+      const int64_t rnt = cdiv(r, p.r_bn_mn);
+      p.du = choose_split(cdiv(T, 128) * rnt, cdiv(d_out, 64), p.sms);
+      if (p.du.splits > 1) p.off_du_part = take((size_t)p.du.splits * T * r * 4);
+      p.off_du = take((size_t)T * r * 2);
+      p.dB = choose_split(cdiv(d_out, 128) * rnt, cdiv(T, 64), p.sms);
+      if (p.dB.splits > 1) p.off_dB_part = take((size_t)p.dB.splits * d_out * r * 4);
+      p.dA = choose_split(cdiv(d_in, 128) * rnt, cdiv(T, 64), p.sms);
+      if (p.dA.splits > 1) p.off_dA_part = take((size_t)p.dA.splits * d_in * r * 4);
+    }
+  } else {
+    if (op == DORA_OP_NORM) {
+      p.off_f32_a = take((size_t)d_out * r * 4);
+      p.off_f32_b = take((size_t)r * r * 4);
+      p.off_f32_c = take((size_t)d_out * r * 4);
+    } else if (op == DORA_OP_FORWARD && T > 0) {
+      p.off_f32_a = take((size_t)T * r * 4);
+      p.off_f32_b = take((size_t)T * d_out * 4);
+    } else if (op == DORA_OP_BACKWARD && T > 0) {
+      p.off_f32_a = take((size_t)T * d_out * 4);
+      p.off_f32_b = take((size_t)cdiv(T, 64) * d_out * 4);
+      p.off_f32_c = take((size_t)T * r * 4);
+    }
+  }
+  p.total = off;
+  return p;
+}
+
+// ------------------------------------------------------------------ checks
+
+static const int64_t kMaxDim = (int64_t)65535 * 128;  // grid.y limit on 128-row tiles
+
+static bool check_desc(const dora_desc_t* d) {
+  if (!d) return set_error("desc is NULL"), false;
+  if (d->dtype != DORA_BF16 && d->dtype != DORA_FP32) return set_error("desc->dtype is not DORA_BF16 or DORA_FP32"), false;
+  if (d->d_out < 1 || d->d_in < 1 || d->r < 1) return set_error("d_out, d_in and r must be >= 1"), false;
+  if (d->d_out > kMaxDim || d->d_in > kMaxDim) return set_error("d_out or d_in too large"), false;
+  if (!std::isfinite(d->s)) return set_error("s is not finite"), false;
+  if (d->dtype == DORA_BF16) {
+    if (d->d_out % 8 || d->d_in % 8 || d->r % 8)
+      return set_error("bf16 layers need d_out, d_in and r to be multiples of 8"), false;
+  }
+  if (d->r > 512) return set_error("r above 512 is not supported"), false;
+  return true;
+}
+
+static bool check_T(int64_t T) {
+  if (T < 0 || T > kMaxDim) return set_error("T out of range"), false;
+  return true;
+}
+
+static bool check_ptr(const void* p, const char* name, size_t align) {
+  if (!p) return set_error(std::string(name) + " is NULL"), false;
+  if (reinterpret_cast<uintptr_t>(p) % align)
+    return set_error(std::string(name) + " is not " + std::to_string(align) + "-byte aligned"), false;
+  return true;
+}
+
+static bool check_opt_ptr(const void* p, const char* name, size_t align) {
+  return p == nullptr || check_ptr(p, name, align);
+}
+
+static size_t tensor_align(const dora_desc_t* d) { return d->dtype == DORA_BF16 ? 16 : 4; }
+
+// The bf16 path runs tcgen05 kernels built for sm_100a only.
+static dora_status_t check_device(const dora_desc_t* d) {
+  if (d->dtype != DORA_BF16) return DORA_OK;
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    set_error("no CUDA device available");
+    return DORA_ECUDA;
+  }
+  if (major != 10 || minor != 0) {
+    set_error("the bf16 path needs an sm_100 (B200) device");
+    return DORA_EUNSUPPORTED;
+  }
+  return DORA_OK;
+}
+
+static dora_status_t check_ws(const Plan& p, const void* ws, size_t ws_bytes) {
+  if (p.total == 0) return DORA_OK;
+  if (!ws) {
+    set_error("workspace is NULL but " + std::to_string(p.total) + " bytes are needed");
+    return DORA_EWORKSPACE;
+  }
+  if (reinterpret_cast<uintptr_t>(ws) % 256) {
+    set_error("workspace is not 256-byte aligned");
+    return DORA_EINVAL;
+  }
+  if (ws_bytes < p.total) {
+    set_error("workspace has " + std::to_string(ws_bytes) + " bytes, needs " + std::to_string(p.total));
+    return DORA_EWORKSPACE;
+  }
+  return DORA_OK;
+}
+
+}  // namespace dora
+
+using namespace dora;
+
+extern "C" {
+
+size_t dora_workspace_size(const dora_desc_t* desc, int64_t T, int op) {
+  if (!check_desc(desc) || !check_T(T) || op < DORA_OP_NORM || op > DORA_OP_BACKWARD) return 0;
+  return make_plan(*desc, T, op).total;
+}
+
+dora_status_t dora_norm(const dora_desc_t* desc, const void* W0, const void* A, const void* B, const float* m,
+                        float* norm_out, float* g_out, float* gm1_out, void* ws, size_t ws_bytes,
+                        dora_stream_t stream) {
+  if (!check_desc(desc)) return DORA_EINVAL;
+  const size_t al = tensor_align(desc);
+  if (!check_ptr(W0, "W0", al) || !check_ptr(A, "A", al) || !check_ptr(B, "B", al) || !check_ptr(m, "m", 4) ||
+      !check_ptr(norm_out, "norm_out", 4) || !check_ptr(g_out, "g_out", 4) || !check_ptr(gm1_out, "gm1_out", 4))
+    return DORA_EINVAL;
+  const Plan p = make_plan(*desc, 0, DORA_OP_NORM);
+  dora_status_t s = check_ws(p, ws, ws_bytes);
+  if (s != DORA_OK) return s;
+  if ((s = check_device(desc)) != DORA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = reinterpret_cast<uint8_t*>(ws);
+  if (desc->dtype == DORA_BF16) return bf16_norm(*desc, p, W0, A, B, m, norm_out, g_out, gm1_out, w, st);
+  return f32_norm(*desc, p, (const float*)W0, (const float*)A, (const float*)B, m, norm_out, g_out, gm1_out, w, st);
+}
+
+dora_status_t dora_forward(const dora_desc_t* desc, int64_t T, const void* x, const void* W0, const void* A,
+                           const void* B, const float* gm1, void* y, void* su_save, void* pre_save, void* ws,
+                           size_t ws_bytes, dora_stream_t stream) {
+  if (!check_desc(desc) || !check_T(T)) return DORA_EINVAL;
+  const size_t al = tensor_align(desc);
+  // Per-token tensors have no elements when T == 0 and may then be NULL.
+  const bool tok = T > 0;
+  if ((tok && !check_ptr(x, "x", al)) || !check_ptr(W0, "W0", al) || !check_ptr(A, "A", al) ||
+      !check_ptr(B, "B", al) || !check_ptr(gm1, "gm1", 16) || (tok && !check_ptr(y, "y", al)) ||
+      !check_opt_ptr(su_save, "su_save", al) || !check_opt_ptr(pre_save, "pre_save", al))
+    return DORA_EINVAL;
+  const Plan p = make_plan(*desc, T, DORA_OP_FORWARD);
+  dora_status_t s = check_ws(p, ws, ws_bytes);
+  if (s != DORA_OK) return s;
+  if ((s = check_device(desc)) != DORA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = reinterpret_cast<uint8_t*>(ws);
+  if (desc->dtype == DORA_BF16) return bf16_forward(*desc, p, T, x, W0, A, B, gm1, y, su_save, pre_save, w, st);
+  return f32_forward(*desc, p, T, (const float*)x, (const float*)W0, (const float*)A, (const float*)B, gm1,
+                     (float*)y, (float*)su_save, (float*)pre_save, w, st);
+}
+
+dora_status_t dora_backward(const dora_desc_t* desc, int64_t T, const void* dy, const void* x, const void* W0,
+                            const void* A, const void* B, const float* norm, const float* g, const void* su_save,
+                            const void* pre_save, float* dm, void* dA, void* dB, void* dx, void* ws,
+                            size_t ws_bytes, dora_stream_t stream) {
+  if (!check_desc(desc) || !check_T(T)) return DORA_EINVAL;
+  const size_t al = tensor_align(desc);
+  // Per-token tensors have no elements when T == 0 and may then be NULL.
+  const bool tok = T > 0;
+  if ((tok && !check_ptr(dy, "dy", al)) || (tok && !check_ptr(x, "x", al)) || !check_ptr(W0, "W0", al) ||
+      !check_ptr(A, "A", al) || !check_ptr(B, "B", al) || !check_ptr(norm, "norm", 4) || !check_ptr(g, "g", 16) ||
+      (tok && !check_ptr(su_save, "su_save", al)) || (tok && !check_ptr(pre_save, "pre_save", al)) ||
+      !check_ptr(dm, "dm", 4) || !check_ptr(dA, "dA", al) || !check_ptr(dB, "dB", al) ||
+      !check_opt_ptr(dx, "dx", al))
+    return DORA_EINVAL;
+  const Plan p = make_plan(*desc, T, DORA_OP_BACKWARD);
+  dora_status_t s = check_ws(p, ws, ws_bytes);
+  if (s != DORA_OK) return s;
+  if ((s = check_device(desc)) != DORA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = reinterpret_cast<uint8_t*>(ws);
+  if (desc->dtype == DORA_BF16)
+    return bf16_backward(*desc, p, T, dy, x, W0, A, B, norm, g, su_save, pre_save, dm, dA, dB, dx, w, st);
+  return f32_backward(*desc, p, T, (const float*)dy, (const float*)x, (const float*)W0, (const float*)A,
+                      (const float*)B, norm, g, (const float*)su_save, (const float*)pre_save, dm, (float*)dA,
+                      (float*)dB, (float*)dx, w, st);
+}
+
+dora_status_t dora_device_status(dora_stream_t stream, unsigned int* flags_out) {
+  if (!flags_out) {
+    set_error("flags_out is NULL");
+    return DORA_EINVAL;
+  }
+  unsigned int v = 0;
+  cudaError_t e = read_and_clear_device_status(reinterpret_cast<cudaStream_t>(stream), &v);
+  if (e != cudaSuccess) return cuda_status(e, "dora_device_status");
+  *flags_out = v;
+  if (v) {
+    set_error("a kernel's bounded wait ran out");
+    return DORA_ETIMEOUT;
+  }
+  return DORA_OK;
+}
+
+const char* dora_last_error(void) { return t_last_error.c_str(); }
+
+int dora_version(void) { return 100; }
+
+}  // extern "C"

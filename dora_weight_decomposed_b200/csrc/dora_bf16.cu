@@ -1,0 +1,647 @@
+// bf16 path of the DoRA layer: tcgen05/TMA GEMMs with the DoRA arithmetic in
+// their epilogues, plus bandwidth-bound SIMT kernels for the compose backward
+// and the small reductions.
+//
+//   dora_norm     Gram G = A A^T (split-K partials -> (s/2) G as bf16 hi + lo), then
+//                 one GEMM  acc = [W0 | B | B] [A | Gs_hi | Gs_lo]^T  whose epilogue forms
+//                 sum_k W0_ik^2 (read from the W0 tiles in shared memory as they
+//                 stream past) + 2 s B_i . acc_i  per row and K split; a finalize
+//                 kernel sums the splits and takes C, g, g - 1.
+//                 2 s B_i . acc_i = 2 s B_i (W0 A^T)_i + s^2 B_i G B_i^T: the cross
+//                 and Gram terms of the factored norm (Scaling DoRA abstract).
+//   dora_forward  su = s x A^T, then  pre = [x | su] [W0 | B]^T  with the
+//                 compose y = pre + gm1 * pre  in the epilogue (one rounding).
+//   dora_backward dz = g * dy and the dm column sums in one streaming pass;
+//                 du = s dz B, dB = dz^T su, dA = du^T x, dx = [dz | du] [W0 ; A].
+#include <algorithm>
+#include <atomic>
+#include <mutex>
+#include <string>
+
+#include "dora_internal.h"
+#include "gemm_sm100.cuh"
+
+namespace dora {
+
+static inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ============================================================== tensor maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Row-major bf16 matrix [rows x cols], leading dimension ld elements.
+struct Mat {
+  const void* ptr = nullptr;
+  int64_t rows = 0, cols = 0, ld = 0;
+};
+
+// Tiles of box_outer rows x 64 columns, 128-byte swizzle, zeros out of bounds.
+static thread_local std::string t_detail;
+
+static bool make_map(CUtensorMap* map, const Mat& m, int box_outer, const char* what) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) {
+    t_detail = "cuTensorMapEncodeTiled unavailable";
+    return false;
+  }
+  if (m.rows <= 0 || m.cols <= 0) {
+    t_detail = std::string(what) + ": empty matrix";
+    return false;
+  }
+  cuuint64_t dims[2] = {(cuuint64_t)m.cols, (cuuint64_t)m.rows};
+  cuuint64_t strides[1] = {(cuuint64_t)m.ld * 2};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_outer};
+  cuuint32_t estr[2] = {1u, 1u};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(m.ptr), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    t_detail = std::string(what) + ": tensor map encode failed (CUresult " + std::to_string((int)r) + ", " +
+               std::to_string(m.rows) + "x" + std::to_string(m.cols) + " ld " + std::to_string(m.ld) + " box " +
+               std::to_string(box_outer) + ")";
+    return false;
+  }
+  return true;
+}
+
+static dora_status_t gemm_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return DORA_OK;
+  set_error(std::string(where) + ": " + cudaGetErrorString(e) + (t_detail.empty() ? "" : " [" + t_detail + "]"));
+  return DORA_ECUDA;
+}
+
+// ============================================================== GEMM launch
+
+struct GemmArgs {
+  Mat a0, a1, b0, b1;  // K-source 0 and (if K1 > 0) 1 of each operand
+  int64_t K0 = 0, K1 = 0;
+  int M = 0, N = 0;
+  Split split;
+  int a1_kwrap = 0;  // see GemmGeom::a1_kwrap
+};
+
+// Raise the kernel's dynamic shared-memory limit once per device; `done` is
+// the caller's own flag word (one per kernel instantiation).
+template <class Kern>
+static cudaError_t set_smem_once(std::atomic<unsigned long long>& done, Kern kern, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (done.load() & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit);
+  return e;
+}
+
+template <class Cfg, class Epi>
+static cudaError_t launch_gemm(const GemmArgs& g, const typename Epi::Params& ep, cudaStream_t st) {
+  CUtensorMap ta0, ta1, tb0, tb1;
+  const int a_box = Cfg::A_MN ? 64 : kBM;
+  const int b_box = Cfg::B_MN ? 64 : Cfg::B_BOX;
+  t_detail.clear();
+  if (!make_map(&ta0, g.a0, a_box, "A source 0") || !make_map(&tb0, g.b0, b_box, "B source 0"))
+    return cudaErrorInvalidValue;
+  const int kb0 = (int)ceil_div(g.K0, kBK);
+  const int kb1 = g.K1 > 0 ? (int)ceil_div(g.K1, kBK) : 0;
+  if (kb1 > 0) {
+    if (!make_map(&ta1, g.a1, a_box, "A source 1") || !make_map(&tb1, g.b1, b_box, "B source 1"))
+      return cudaErrorInvalidValue;
+  } else {
+    ta1 = ta0;
+    tb1 = tb0;
+  }
+  GemmGeom geom{g.M, g.N, kb0, kb1, g.split.kb_per_split, g.a1_kwrap};
+  dim3 grid((unsigned)ceil_div(g.N, Cfg::BN), (unsigned)ceil_div(g.M, kBM), (unsigned)g.split.splits);
+  auto kern = gemm_sm100_kernel<Cfg, Epi>;
+  static std::atomic<unsigned long long> smem_set{0};
+  cudaError_t e = set_smem_once(smem_set, kern, Cfg::SMEM_BYTES);
+  if (e != cudaSuccess) {
+    t_detail = "shared-memory attribute (" + std::to_string(Cfg::SMEM_BYTES) + " bytes)";
+    return e;
+  }
+  kern<<<grid, kGemmThreads, Cfg::SMEM_BYTES, st>>>(ta0, ta1, tb0, tb1, geom, ep);
+  e = cudaGetLastError();
+  if (e != cudaSuccess)
+    t_detail = "launch grid (" + std::to_string(grid.x) + "," + std::to_string(grid.y) + "," +
+               std::to_string(grid.z) + ") smem " + std::to_string(Cfg::SMEM_BYTES);
+  return e;
+}
+
+// Tile width for the narrow (N = r) GEMMs with K-major B.
+static int bn_skinny(int64_t r) { return r <= 16 ? 16 : r <= 32 ? 32 : r <= 64 ? 64 : 128; }
+
+template <bool A_MN, bool B_MN, class Epi>
+static cudaError_t gemm_bn(int bn, const GemmArgs& g, const typename Epi::Params& ep, cudaStream_t st) {
+  if constexpr (!B_MN) {
+    if (bn == 16) return launch_gemm<GemmCfg<16, A_MN, B_MN>, Epi>(g, ep, st);
+    if (bn == 32) return launch_gemm<GemmCfg<32, A_MN, B_MN>, Epi>(g, ep, st);
+  }
+  if (bn == 64) return launch_gemm<GemmCfg<64, A_MN, B_MN>, Epi>(g, ep, st);
+  if (bn == 128) return launch_gemm<GemmCfg<128, A_MN, B_MN>, Epi>(g, ep, st);
+  return cudaErrorInvalidValue;
+}
+
+// ============================================================== DoRA epilogues
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4& w, float* f) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+// Factored-norm epilogue. For each row i of W0 and each K split z:
+//   part[z][i] = sum_{k in split, k < d_in} W0_ik^2 + 2 s sum_n B_in acc_in
+// with acc = [W0 | B | B] [A | (s/2) G_hi | (s/2) G_lo]^T over the split's k-blocks.
+struct EpiNorm {
+  struct Params {
+    const __nv_bfloat16* B;  // [d_out x r]
+    int r;
+    float two_s;
+    float* part;             // [splits][d_out]
+    int d_out;
+  };
+  struct RowState {
+    float ss = 0.f;
+  };
+  static constexpr bool kReadsA = true;
+  // row_ptr: this thread's 128-byte row of the W0 tile (swizzle only permutes
+  // 16-byte chunks inside the row, which a sum of squares does not see).
+  __device__ static void on_a_stage(const Params&, RowState& st, const uint8_t* row_ptr, bool src1) {
+    if (src1) return;
+    const uint4* p = reinterpret_cast<const uint4*>(row_ptr);
+    float acc = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float f[8];
+      unpack_bf16x8(p[j], f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc = fmaf(f[i], f[i], acc);
+    }
+    st.ss += acc;
+  }
+  template <int BN>
+  __device__ static void run(const Params& p, RowState& st, const EpiCtx& c, const GemmGeom& g) {
+    const bool row_ok = c.m < g.M;
+    const __nv_bfloat16* brow = p.B + (long long)(row_ok ? c.m : 0) * p.r;
+    float dot = 0.f;
+    for_each_acc_chunk<BN>(c, [&](int col, float* v) {
+      if (!row_ok) return;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int n = col + 8 * j;
+        if (n < p.r) {
+          float b[8];
+          unpack_bf16x8(*reinterpret_cast<const uint4*>(brow + n), b);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) dot = fmaf(b[i], v[8 * j + i], dot);
+        }
+      }
+    });
+    if (row_ok) p.part[(long long)c.split * p.d_out + c.m] = fmaf(p.two_s, dot, st.ss);
+  }
+};
+
+// Near-unity compose: y = pre + gm1[n] * pre (fp32, rounded once), pre optional.
+struct EpiCompose {
+  struct Params {
+    __nv_bfloat16* y;
+    __nv_bfloat16* pre;  // may be null
+    const float* gm1;
+    long long ldo;
+  };
+  using RowState = NoRowState;
+  static constexpr bool kReadsA = false;
+  __device__ static void on_a_stage(const Params&, RowState&, const uint8_t*, bool) {}
+  template <int BN>
+  __device__ static void run(const Params& p, RowState&, const EpiCtx& c, const GemmGeom& g) {
+    const bool row_ok = c.m < g.M;
+    for_each_acc_chunk<BN>(c, [&](int col, float* v) {
+      if (!row_ok) return;
+      const int n = c.n0 + col;
+      __nv_bfloat16* yrow = p.y + (long long)c.m * p.ldo + n;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (n + 8 * j < g.N) {
+          const float4 ga = __ldg(reinterpret_cast<const float4*>(p.gm1 + n + 8 * j));
+          const float4 gb = __ldg(reinterpret_cast<const float4*>(p.gm1 + n + 8 * j + 4));
+          const float gm[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+          float o[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) o[i] = fmaf(gm[i], v[8 * j + i], v[8 * j + i]);
+          store_bf16x8(yrow + 8 * j, o);
+          if (p.pre) store_bf16x8(p.pre + (long long)c.m * p.ldo + n + 8 * j, v + 8 * j);
+        }
+      }
+    });
+  }
+};
+
+template <int BN>
+static cudaError_t norm_gemm_bn(const GemmArgs& g, const EpiNorm::Params& ep, cudaStream_t st) {
+  return launch_gemm<GemmCfg<BN, false, false>, EpiNorm>(g, ep, st);
+}
+
+static int bn_norm(int64_t r) {
+  return r <= 16 ? 16 : r <= 32 ? 32 : r <= 64 ? 64 : r <= 128 ? 128 : r <= 256 ? 256 : r <= 384 ? 384 : 512;
+}
+
+static cudaError_t norm_gemm(int bn, const GemmArgs& g, const EpiNorm::Params& ep, cudaStream_t st) {
+  switch (bn) {
+    case 16: return norm_gemm_bn<16>(g, ep, st);
+    case 32: return norm_gemm_bn<32>(g, ep, st);
+    case 64: return norm_gemm_bn<64>(g, ep, st);
+    case 128: return norm_gemm_bn<128>(g, ep, st);
+    case 256: return norm_gemm_bn<256>(g, ep, st);
+    case 384: return norm_gemm_bn<384>(g, ep, st);
+    case 512: return norm_gemm_bn<512>(g, ep, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+// ============================================================== SIMT kernels
+
+// out = alpha * sum_z part[z] (split order fixed), bf16; out[n][m] if transpose.
+__global__ void reduce_splits_bf16_kernel(const float* __restrict__ part, int splits, long long split_stride,
+                                          int M, int N, float alpha, __nv_bfloat16* __restrict__ out,
+                                          long long ldo, int transpose) {
+  const int ng = N / 4;
+  const long long total = (long long)M * ng;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    int m, n;
+    if (!transpose) {
+      m = (int)(i / ng);
+      n = (int)(i % ng) * 4;
+    } else {
+      n = (int)(i / M) * 4;
+      m = (int)(i % M);
+    }
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int z = 0; z < splits; ++z) {
+      const float4 v = *reinterpret_cast<const float4*>(part + z * split_stride + (long long)m * N + n);
+      a.x += v.x;
+      a.y += v.y;
+      a.z += v.z;
+      a.w += v.w;
+    }
+    const float o[4] = {alpha * a.x, alpha * a.y, alpha * a.z, alpha * a.w};
+    if (!transpose) {
+      __nv_bfloat162 h[2] = {__floats2bfloat162_rn(o[0], o[1]), __floats2bfloat162_rn(o[2], o[3])};
+      *reinterpret_cast<uint2*>(out + (long long)m * ldo + n) = *reinterpret_cast<const uint2*>(h);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) out[(long long)(n + j) * ldo + m] = __float2bfloat16_rn(o[j]);
+    }
+  }
+}
+
+// Gram finalize: x = (s/2) sum_z part[z] in fp32, written as two bf16 halves
+// Gs2[n] = [hi(x_n,0..r-1), 0 .. | lo(x_n,0..r-1), 0 ..] with rp columns each,
+// hi = bf16(x) and lo = bf16(x - hi), so hi + lo carries x to about 2^-17.
+__global__ void gram_finalize_kernel(const float* __restrict__ part, int splits, int r, int rp, float half_s,
+                                     __nv_bfloat16* __restrict__ gs2) {
+  const long long total = (long long)r * 2 * rp;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int n = (int)(i / (2 * rp));
+    const int k = (int)(i % (2 * rp));
+    const bool lo = k >= rp;
+    const int c = lo ? k - rp : k;
+    float v = 0.f;
+    if (c < r) {
+      float x = 0.f;
+      for (int z = 0; z < splits; ++z) x += part[(long long)z * r * r + (long long)n * r + c];
+      x *= half_s;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+      v = lo ? x - __bfloat162float(hi) : x;
+    }
+    gs2[i] = __float2bfloat16_rn(v);
+  }
+}
+
+// C = sqrt(max(0, sum of partials)), g = m / C, gm1 = (m - C) / C.
+__global__ void norm_finalize_kernel(const float* __restrict__ part, int nparts, int d_out,
+                                     const float* __restrict__ m, float* __restrict__ C, float* __restrict__ g,
+                                     float* __restrict__ gm1) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= d_out) return;
+  float sq = 0.f;
+  for (int z = 0; z < nparts; ++z) sq += part[(long long)z * d_out + i];
+  const float c = sqrtf(fmaxf(sq, 0.f));
+  const float mi = m[i];
+  C[i] = c;
+  g[i] = mi / c;
+  gm1[i] = (mi - c) / c;
+}
+
+// Compose backward, one streaming pass over [T x d_out]:
+//   dz[t][i] = g_i * dy[t][i]   (bf16)
+//   part[rb][i] = sum over the row block's t of dy[t][i] * pre[t][i]
+// Block: 256 threads, 64 columns x kCbRows rows. Lane = (row offset 0..3,
+// 8-column vector 0..7), so each warp access covers 4 full 128-byte rows; the
+// per-column sums are combined over the 4 row lanes with shuffles, then over
+// the 8 warps in shared memory.
+constexpr int kCbRows = 256;
+
+__global__ void __launch_bounds__(256) compose_bwd_bf16_kernel(const __nv_bfloat16* __restrict__ dy,
+                                                               const __nv_bfloat16* __restrict__ pre,
+                                                               const float* __restrict__ g,
+                                                               __nv_bfloat16* __restrict__ dz,
+                                                               float* __restrict__ part, int T, int d_out) {
+  __shared__ float red[8][64];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cv = lane & 7, ro = lane >> 3;
+  const int col = blockIdx.x * 64 + cv * 8;
+  const bool col_ok = col < d_out;
+  const int t0 = blockIdx.y * kCbRows;
+  const int t1 = min(T, t0 + kCbRows);
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+  if (col_ok) {
+    const float4 ga = __ldg(reinterpret_cast<const float4*>(g + col));
+    const float4 gb = __ldg(reinterpret_cast<const float4*>(g + col + 4));
+    const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+#pragma unroll 4
+    for (int t = t0 + warp * 4 + ro; t < t1; t += 32) {
+      const size_t off = (size_t)t * d_out + col;
+      const uint4 a = __ldcs(reinterpret_cast<const uint4*>(dy + off));
+      const uint4 b = __ldcs(reinterpret_cast<const uint4*>(pre + off));
+      float fa[8], fb[8], z[8];
+      unpack_bf16x8(a, fa);
+      unpack_bf16x8(b, fb);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        acc[j] = fmaf(fa[j], fb[j], acc[j]);
+        z[j] = gv[j] * fa[j];
+      }
+      store_bf16x8(dz + off, z);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], 8);
+    acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], 16);
+  }
+  if (ro == 0) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) red[warp][cv * 8 + j] = acc[j];
+  }
+  __syncthreads();
+  if (threadIdx.x < 64) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += red[w][threadIdx.x];
+    const int c = blockIdx.x * 64 + threadIdx.x;
+    if (c < d_out) part[(size_t)blockIdx.y * d_out + c] = s;
+  }
+}
+
+// dm_i = (sum over row blocks of part[rb][i]) / C_i.
+__global__ void dm_finalize_kernel(const float* __restrict__ part, int nparts, int d_out,
+                                   const float* __restrict__ C, float* __restrict__ dm) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= d_out) return;
+  float s = 0.f;
+  for (int z = 0; z < nparts; ++z) s += part[(long long)z * d_out + i];
+  dm[i] = s / C[i];
+}
+
+static cudaError_t reduce_splits(const float* part, const Split& sp, long long split_stride, int M, int N,
+                                 float alpha, __nv_bfloat16* out, long long ldo, bool transpose, cudaStream_t st) {
+  const long long total = (long long)M * (N / 4);
+  const int threads = 256;
+  const long long blocks = std::min<long long>(ceil_div(total, threads), 148LL * 16);
+  reduce_splits_bf16_kernel<<<(unsigned)std::max<long long>(blocks, 1), threads, 0, st>>>(
+      part, sp.splits, split_stride, M, N, alpha, out, ldo, transpose ? 1 : 0);
+  return cudaGetLastError();
+}
+
+// Narrow GEMM (N = r) with an alpha-scaled bf16 result: direct store when the
+// K loop is not split, else fp32 partials summed by reduce_splits.
+template <bool A_MN, bool B_MN>
+static cudaError_t narrow_gemm(int bn, const GemmArgs& g, float alpha, __nv_bfloat16* out, long long ldo,
+                               bool transpose, float* part, cudaStream_t st) {
+  if (g.split.splits == 1) {
+    EpiStoreBF16::Params p{out, ldo, alpha, transpose ? 1 : 0};
+    return gemm_bn<A_MN, B_MN, EpiStoreBF16>(bn, g, p, st);
+  }
+  const long long sstride = (long long)g.M * g.N;
+  EpiPartialF32::Params p{part, g.N, sstride};
+  cudaError_t e = gemm_bn<A_MN, B_MN, EpiPartialF32>(bn, g, p, st);
+  if (e != cudaSuccess) return e;
+  return reduce_splits(part, g.split, sstride, g.M, g.N, alpha, out, ldo, transpose, st);
+}
+
+// ============================================================== operations
+
+dora_status_t bf16_norm(const dora_desc_t& d, const Plan& p, const void* W0, const void* A, const void* B,
+                        const float* m, float* C, float* g, float* gm1, uint8_t* ws, cudaStream_t st) {
+  const int r = (int)d.r, d_in = (int)d.d_in, d_out = (int)d.d_out;
+  float* gram_part = reinterpret_cast<float*>(ws + p.off_gram_part);
+  __nv_bfloat16* gs = reinterpret_cast<__nv_bfloat16*>(ws + p.off_gs);
+  float* norm_part = reinterpret_cast<float*>(ws + p.off_norm_part);
+
+  // Gram G = A A^T in fp32 partials, then (s/2) G as bf16 hi and lo halves.
+  const int rp = (int)ceil_div(r, kBK) * kBK;
+  GemmArgs ga;
+  ga.a0 = Mat{A, r, d_in, d_in};
+  ga.b0 = ga.a0;
+  ga.K0 = d_in;
+  ga.M = r;
+  ga.N = r;
+  ga.split = p.gram;
+  {
+    const long long sstride = (long long)r * r;
+    EpiPartialF32::Params pp{gram_part, r, sstride};
+    cudaError_t e = gemm_bn<false, false, EpiPartialF32>(bn_skinny(r), ga, pp, st);
+    if (e != cudaSuccess) return gemm_status(e, "dora_norm: Gram");
+    const long long total = (long long)r * 2 * rp;
+    gram_finalize_kernel<<<(unsigned)std::min<long long>(ceil_div(total, 256), 2048), 256, 0, st>>>(
+        gram_part, p.gram.splits, r, rp, 0.5f * d.s, gs);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_status(e, "dora_norm: Gram finalize");
+  }
+
+  // acc = [W0 | B | B] [A | Gs_hi | Gs_lo]^T with the factored-norm epilogue.
+  GemmArgs na;
+  na.a0 = Mat{W0, d_out, d_in, d_in};
+  na.a1 = Mat{B, d_out, r, r};
+  na.b0 = Mat{A, r, d_in, d_in};
+  na.b1 = Mat{gs, r, 2 * rp, 2 * rp};
+  na.K0 = d_in;
+  na.K1 = 2 * rp;
+  na.a1_kwrap = rp;
+  na.M = d_out;
+  na.N = r;
+  na.split = p.norm;
+  EpiNorm::Params np{reinterpret_cast<const __nv_bfloat16*>(B), r, 2.0f * d.s, norm_part, d_out};
+  cudaError_t e = norm_gemm(bn_norm(r), na, np, st);
+  if (e != cudaSuccess) return gemm_status(e, "dora_norm: factored norm GEMM");
+
+  norm_finalize_kernel<<<(unsigned)ceil_div(d_out, 256), 256, 0, st>>>(norm_part, p.norm.splits, d_out, m, C, g,
+                                                                        gm1);
+  return cuda_status(cudaGetLastError(), "dora_norm: finalize");
+}
+
+dora_status_t bf16_forward(const dora_desc_t& d, const Plan& p, int64_t T, const void* x, const void* W0,
+                           const void* A, const void* B, const float* gm1, void* y, void* su_save,
+                           void* pre_save, uint8_t* ws, cudaStream_t st) {
+  if (T == 0) return DORA_OK;
+  const int r = (int)d.r, d_in = (int)d.d_in, d_out = (int)d.d_out, Ti = (int)T;
+  __nv_bfloat16* su = su_save ? reinterpret_cast<__nv_bfloat16*>(su_save)
+                              : reinterpret_cast<__nv_bfloat16*>(ws + p.off_su);
+
+  // su = s x A^T
+  GemmArgs ua;
+  ua.a0 = Mat{x, Ti, d_in, d_in};
+  ua.b0 = Mat{A, r, d_in, d_in};
+  ua.K0 = d_in;
+  ua.M = Ti;
+  ua.N = r;
+  ua.split = p.u;
+  cudaError_t e = narrow_gemm<false, false>(p.u_bn, ua, d.s, su, r, false,
+                                            reinterpret_cast<float*>(ws + p.off_u_part), st);
+  if (e != cudaSuccess) return gemm_status(e, "dora_forward: LoRA down projection");
+
+  // pre = [x | su] [W0 | B]^T, y = pre + gm1 * pre
+  GemmArgs ba;
+  ba.a0 = Mat{x, Ti, d_in, d_in};
+  ba.a1 = Mat{su, Ti, r, r};
+  ba.b0 = Mat{W0, d_out, d_in, d_in};
+  ba.b1 = Mat{B, d_out, r, r};
+  ba.K0 = d_in;
+  ba.K1 = r;
+  ba.M = Ti;
+  ba.N = d_out;
+  ba.split.splits = 1;
+  ba.split.kb_per_split = (int)(ceil_div(d_in, kBK) + ceil_div(r, kBK));
+  EpiCompose::Params cp{reinterpret_cast<__nv_bfloat16*>(y), reinterpret_cast<__nv_bfloat16*>(pre_save), gm1,
+                        d_out};
+  e = launch_gemm<GemmCfg<256, false, false>, EpiCompose>(ba, cp, st);
+  return gemm_status(e, "dora_forward: base GEMM with compose");
+}
+
+dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, const void* dy, const void* x,
+                            const void* W0, const void* A, const void* B, const float* C, const float* g,
+                            const void* su, const void* pre, float* dm, void* dA, void* dB, void* dx,
+                            uint8_t* ws, cudaStream_t st) {
+  const int r = (int)d.r, d_in = (int)d.d_in, d_out = (int)d.d_out, Ti = (int)T;
+  if (T == 0) {
+    cudaError_t e = cudaMemsetAsync(dm, 0, sizeof(float) * d_out, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dA, 0, 2 * (size_t)r * d_in, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dB, 0, 2 * (size_t)d_out * r, st);
+    return cuda_status(e, "dora_backward: empty batch");
+  }
+  __nv_bfloat16* dz = reinterpret_cast<__nv_bfloat16*>(ws + p.off_dz);
+  float* dm_part = reinterpret_cast<float*>(ws + p.off_dm_part);
+  __nv_bfloat16* du = reinterpret_cast<__nv_bfloat16*>(ws + p.off_du);
+
+  // dz = g * dy, dm = sum_t dy * pre / C
+  {
+    dim3 grid((unsigned)ceil_div(d_out, 64), (unsigned)p.dm_rowblocks);
+    compose_bwd_bf16_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(dy),
+                                                  reinterpret_cast<const __nv_bfloat16*>(pre), g, dz, dm_part,
+                                                  Ti, d_out);
+    dm_finalize_kernel<<<(unsigned)ceil_div(d_out, 256), 256, 0, st>>>(dm_part, p.dm_rowblocks, d_out, C, dm);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_status(e, "dora_backward: compose backward");
+  }
+  // du = s dz B  (B read MN-major: K = d_out rows, N = r contiguous)
+  {
+    GemmArgs a;
+    a.a0 = Mat{dz, Ti, d_out, d_out};
+    a.b0 = Mat{B, d_out, r, r};
+    a.K0 = d_out;
+    a.M = Ti;
+    a.N = r;
+    a.split = p.du;
+    cudaError_t e = narrow_gemm<false, true>(p.r_bn_mn, a, d.s, du, r, false,
+                                             reinterpret_cast<float*>(ws + p.off_du_part), st);
+    if (e != cudaSuccess) return gemm_status(e, "dora_backward: du");
+  }
+  // dB = dz^T su  (both token-major: K = T)
+  {
+    GemmArgs a;
+    a.a0 = Mat{dz, Ti, d_out, d_out};
+    a.b0 = Mat{su, Ti, r, r};
+    a.K0 = Ti;
+    a.M = d_out;
+    a.N = r;
+    a.split = p.dB;
+    cudaError_t e = narrow_gemm<true, true>(p.r_bn_mn, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dB), r, false,
+                                            reinterpret_cast<float*>(ws + p.off_dB_part), st);
+    if (e != cudaSuccess) return gemm_status(e, "dora_backward: dB");
+  }
+  // dA^T = x^T du, stored transposed into dA [r x d_in]
+  {
+    GemmArgs a;
+    a.a0 = Mat{x, Ti, d_in, d_in};
+    a.b0 = Mat{du, Ti, r, r};
+    a.K0 = Ti;
+    a.M = d_in;
+    a.N = r;
+    a.split = p.dA;
+    cudaError_t e = narrow_gemm<true, true>(p.r_bn_mn, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dA), d_in, true,
+                                            reinterpret_cast<float*>(ws + p.off_dA_part), st);
+    if (e != cudaSuccess) return gemm_status(e, "dora_backward: dA");
+  }
+  // dx = [dz | du] [W0 ; A]  (W0 and A read MN-major: K rows, N = d_in contiguous)
+  if (dx) {
+    GemmArgs a;
+    a.a0 = Mat{dz, Ti, d_out, d_out};
+    a.a1 = Mat{du, Ti, r, r};
+    a.b0 = Mat{W0, d_out, d_in, d_in};
+    a.b1 = Mat{A, r, d_in, d_in};
+    a.K0 = d_out;
+    a.K1 = r;
+    a.M = Ti;
+    a.N = d_in;
+    a.split.splits = 1;
+    a.split.kb_per_split = (int)(ceil_div(d_out, kBK) + ceil_div(r, kBK));
+    EpiStoreBF16::Params sp{reinterpret_cast<__nv_bfloat16*>(dx), d_in, 1.0f, 0};
+    cudaError_t e = launch_gemm<GemmCfg<256, false, true>, EpiStoreBF16>(a, sp, st);
+    if (e != cudaSuccess) return gemm_status(e, "dora_backward: dx");
+  }
+  return DORA_OK;
+}
+
+}  // namespace dora
+
+namespace dora {
+
+cudaError_t read_and_clear_device_status(cudaStream_t st, unsigned int* out) {
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return e;
+  unsigned int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v));
+  if (e != cudaSuccess) return e;
+  if (v) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero));
+  }
+  *out = v;
+  return e;
+}
+
+}  // namespace dora

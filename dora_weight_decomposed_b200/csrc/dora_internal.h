@@ -1,0 +1,78 @@
+// Internal declarations shared by the C ABI (dora_api.cu) and the bf16 / fp32
+// implementations. Nothing here is exported.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <string>
+
+#include <cuda_runtime.h>
+
+#include "../../include/dora.h"
+
+namespace dora {
+
+// Workspace plan: every offset a call will use, computed from (desc, T, op)
+// and the device's SM count alone, so dora_workspace_size() and the call agree.
+struct Split {
+  int splits = 1;
+  int kb_per_split = 0;
+};
+
+struct Plan {
+  int sms = 148;
+  // norm
+  Split gram, norm;
+  size_t off_gram_part = 0, off_gs = 0, off_norm_part = 0;
+  // forward
+  Split u;
+  int u_bn = 0;
+  size_t off_u_part = 0, off_su = 0;
+  // backward
+  int dm_rowblocks = 0;
+  Split du, dB, dA;
+  int r_bn_mn = 0;
+  size_t off_dz = 0, off_dm_part = 0, off_du_part = 0, off_du = 0, off_dB_part = 0, off_dA_part = 0;
+  // fp32 path scratch
+  size_t off_f32_a = 0, off_f32_b = 0, off_f32_c = 0;
+  size_t total = 0;
+};
+
+int device_sm_count();
+Plan make_plan(const dora_desc_t& d, int64_t T, int op);
+
+// Thread-local error message for dora_last_error().
+void set_error(const std::string& msg);
+
+// Status word written by kernels whose bounded waits ran out.
+cudaError_t read_and_clear_device_status(cudaStream_t st, unsigned int* out);
+
+// bf16 path (tcgen05 / TMA kernels)
+dora_status_t bf16_norm(const dora_desc_t& d, const Plan& p, const void* W0, const void* A, const void* B,
+                        const float* m, float* C, float* g, float* gm1, uint8_t* ws, cudaStream_t st);
+dora_status_t bf16_forward(const dora_desc_t& d, const Plan& p, int64_t T, const void* x, const void* W0,
+                           const void* A, const void* B, const float* gm1, void* y, void* su_save,
+                           void* pre_save, uint8_t* ws, cudaStream_t st);
+dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, const void* dy, const void* x,
+                            const void* W0, const void* A, const void* B, const float* C, const float* g,
+                            const void* su, const void* pre, float* dm, void* dA, void* dB, void* dx,
+                            uint8_t* ws, cudaStream_t st);
+
+// fp32 path (SIMT kernels)
+dora_status_t f32_norm(const dora_desc_t& d, const Plan& p, const float* W0, const float* A, const float* B,
+                       const float* m, float* C, float* g, float* gm1, uint8_t* ws, cudaStream_t st);
+dora_status_t f32_forward(const dora_desc_t& d, const Plan& p, int64_t T, const float* x, const float* W0,
+                          const float* A, const float* B, const float* gm1, float* y, float* su_save,
+                          float* pre_save, uint8_t* ws, cudaStream_t st);
+dora_status_t f32_backward(const dora_desc_t& d, const Plan& p, int64_t T, const float* dy, const float* x,
+                           const float* W0, const float* A, const float* B, const float* C, const float* g,
+                           const float* su, const float* pre, float* dm, float* dA, float* dB, float* dx,
+                           uint8_t* ws, cudaStream_t st);
+
+inline dora_status_t cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return DORA_OK;
+  set_error(std::string(where) + ": " + cudaGetErrorString(e));
+  return DORA_ECUDA;
+}
+
+}  // namespace dora

@@ -1,0 +1,341 @@
+// Warp-specialised tcgen05 GEMM core for sm_100a.
+//
+//   D[M x N] = sum over k of Aop[m, k] * Bop[n, k]      (fp32 accumulator in TMEM)
+//
+// Aop is 128 rows per CTA, Bop is BN rows per CTA, K is streamed in blocks of
+// 64 bf16 (one 128-byte swizzle row) through a STAGES-deep shared-memory ring
+// filled by TMA. Either operand may be stored K-major (rows of K contiguous) or
+// MN-major (rows of M/N contiguous, e.g. a token-major tensor used with K = T).
+// K may come from two sources back to back (source 0 then source 1, e.g.
+// [x | s*u] against [W0 | B]); each source has its own tensor maps. Source 1
+// of A may be re-read cyclically (a1_kwrap) to pair one A block with several
+// B blocks, e.g. [B | B] against [G_hi | G_lo].
+// blockIdx = (n tile, m tile, K split).
+//
+// Warp roles (192 threads):
+//   warp 0     one lane issues the TMA loads for each stage
+//   warp 1     allocates TMEM; one lane issues tcgen05.mma and commits
+//   warps 2-5  epilogue: warp w owns TMEM lanes 32*(w%4) .. +31 (= tile rows);
+//              an epilogue may also read each A stage (kReadsA) before it is
+//              released, which the norm uses for the row sums of squares.
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace dora {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kGemmThreads = 192;
+constexpr int kSmemBudget = 200 * 1024;
+
+struct GemmGeom {
+  int M;             // valid output rows
+  int N;             // valid output columns
+  int kb0;           // k-blocks taken from source 0
+  int kb1;           // k-blocks taken from source 1
+  int kb_per_split;  // k-blocks per blockIdx.z
+  int a1_kwrap;      // > 0: source-1 A coordinates wrap modulo this many K elements
+};
+
+template <int BN_, bool A_MN_, bool B_MN_>
+struct GemmCfg {
+  static constexpr int BN = BN_;
+  static constexpr bool A_MN = A_MN_;
+  static constexpr bool B_MN = B_MN_;
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 512, "BN");
+  static_assert(!B_MN || BN % 64 == 0, "MN-major B tiles are whole 64-wide swizzle chunks");
+  static_assert(BN <= 128 || BN % 128 == 0, "BN above 128 must be a multiple of 128");
+  static constexpr int A_BYTES = kBM * kBK * 2;
+  static constexpr int B_BYTES = BN * kBK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES_RAW = kSmemBudget / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static_assert(STAGES >= 2, "stages");
+  static constexpr int TMEM_COLS = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : BN <= 256 ? 256 : 512;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+  static constexpr int MMA_N0 = BN <= 256 ? BN : 256;
+  static constexpr int MMA_N1 = BN <= 256 ? 0 : BN - 256;
+  // TMA boxes: K-major B uses boxes of B_BOX rows; MN-major uses 64x64 chunks.
+  static constexpr int B_BOX = B_MN ? 64 : (BN <= 128 ? BN : 128);
+  static constexpr int B_LOADS = BN / B_BOX;
+};
+
+struct EpiCtx {
+  uint32_t taddr;  // TMEM address of this warp's lane quarter, column 0
+  int row;         // row within the tile (0..127) owned by this thread
+  int m;           // global output row
+  int n0;          // first global output column of the tile
+  int split;       // blockIdx.z
+  bool has_acc;    // false when this split had no k-blocks (accumulator never written)
+};
+
+// 16-column TMEM load (for tiles whose width is an odd multiple of 16).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  tmem_ld_wait();
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Visit the thread's accumulator row in chunks of 32 columns: f(col, v[32]).
+// A trailing 16-wide chunk is zero-padded to 32. Warp-collective.
+template <int BN, class F>
+__device__ __forceinline__ void for_each_acc_chunk(const EpiCtx& c, F&& f) {
+#pragma unroll 1
+  for (int col = 0; col < BN; col += 32) {
+    float v[32];
+    if (BN - col >= 32) {
+      if (c.has_acc) {
+        tmem_ld32(c.taddr + col, v);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+      }
+    } else {
+      if (c.has_acc) {
+        tmem_ld16(c.taddr + col, v);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 16; i < 32; ++i) v[i] = 0.f;
+    }
+    f(col, v);
+  }
+}
+
+template <class Cfg, class Epi>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_sm100_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tA1,
+                      const __grid_constant__ CUtensorMap tB0, const __grid_constant__ CUtensorMap tB1,
+                      const GemmGeom geom, const typename Epi::Params ep) {
+  constexpr int STAGES = Cfg::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accf = empty + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_tile = blockIdx.x;
+  const int m_tile = blockIdx.y;
+  const int split = blockIdx.z;
+  const int kb_total = geom.kb0 + geom.kb1;
+  const int kb_begin = split * geom.kb_per_split;
+  const int kb_end = min(kb_total, kb_begin + geom.kb_per_split);
+  const int nkb = kb_end > kb_begin ? kb_end - kb_begin : 0;
+
+  if (threadIdx.x == 0) {
+#pragma unroll 1
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1 + (Epi::kReadsA ? 4 : 0));
+    }
+    mbar_init(accf, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tA0);
+    prefetch_tmap(&tB0);
+    if (geom.kb1 > 0) {
+      prefetch_tmap(&tA1);
+      prefetch_tmap(&tB1);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+#pragma unroll 1
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % STAGES;
+        const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+        if (!mbar_wait(&empty[s], ph ^ 1u)) break;
+        uint8_t* sa = smem + s * Cfg::STAGE_BYTES;
+        uint8_t* sb = sa + Cfg::A_BYTES;
+        mbar_arrive_expect_tx(&full[s], Cfg::STAGE_BYTES);
+        const int kb = kb_begin + i;
+        const bool src1 = kb >= geom.kb0;
+        const int k0 = (src1 ? kb - geom.kb0 : kb) * kBK;
+        const int k0a = (src1 && geom.a1_kwrap > 0) ? k0 % geom.a1_kwrap : k0;
+        const CUtensorMap* ta = src1 ? &tA1 : &tA0;
+        const CUtensorMap* tb = src1 ? &tB1 : &tB0;
+        const int m0 = m_tile * kBM;
+        const int n0 = n_tile * Cfg::BN;
+        if (!Cfg::A_MN) {
+          tma_load_2d(sa, ta, &full[s], k0a, m0);
+        } else {
+          tma_load_2d(sa, ta, &full[s], m0, k0a);
+          tma_load_2d(sa + 8192, ta, &full[s], m0 + 64, k0a);
+        }
+#pragma unroll
+        for (int j = 0; j < Cfg::B_LOADS; ++j) {
+          if (!Cfg::B_MN)
+            tma_load_2d(sb + j * Cfg::B_BOX * 128, tb, &full[s], k0, n0 + j * Cfg::B_BOX);
+          else
+            tma_load_2d(sb + j * 8192, tb, &full[s], n0 + j * 64, k0);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc0 = idesc_bf16_f32(kBM, Cfg::MMA_N0, Cfg::A_MN, Cfg::B_MN);
+      constexpr uint32_t idesc1 = idesc_bf16_f32(kBM, Cfg::MMA_N1 > 0 ? Cfg::MMA_N1 : 16, Cfg::A_MN, Cfg::B_MN);
+      // Per 16-wide K step: K-major advances 32 bytes inside the swizzle row,
+      // MN-major advances 16 rows of 128 bytes.
+      constexpr uint32_t a_kstep = Cfg::A_MN ? 2048u : 32u;
+      constexpr uint32_t b_kstep = Cfg::B_MN ? 2048u : 32u;
+      constexpr uint32_t a_lbo = Cfg::A_MN ? 8192u : 16u;
+      constexpr uint32_t b_lbo = Cfg::B_MN ? 8192u : 16u;
+      // Offset of the second MMA's B rows (columns 256..): 256 K-major rows or 4 MN-major chunks.
+      constexpr uint32_t b_half = Cfg::B_MN ? 4u * 8192u : 256u * 128u;
+#pragma unroll 1
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % STAGES;
+        const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+        if (!mbar_wait(&full[s], ph)) break;
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + s * Cfg::STAGE_BYTES);
+        const uint32_t sb = sa + Cfg::A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(sa + kk * a_kstep, a_lbo, 1024u);
+          const uint64_t bd0 = sdesc_sw128(sb + kk * b_kstep, b_lbo, 1024u);
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+          umma_bf16(tmem, ad, bd0, idesc0, acc);
+          if (Cfg::MMA_N1 > 0) {
+            const uint64_t bd1 = sdesc_sw128(sb + b_half + kk * b_kstep, b_lbo, 1024u);
+            umma_bf16(tmem + 256u, ad, bd1, idesc1, acc);
+          }
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(accf);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    typename Epi::RowState st{};
+    if (Epi::kReadsA) {
+#pragma unroll 1
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % STAGES;
+        const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+        if (!mbar_wait(&full[s], ph)) break;
+        const int kb = kb_begin + i;
+        Epi::on_a_stage(ep, st, smem + s * Cfg::STAGE_BYTES + row * 128, kb >= geom.kb0);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
+    }
+    mbar_wait(accf, 0);
+    tc_fence_after();
+    EpiCtx c;
+    c.taddr = tmem + ((uint32_t)(q * 32) << 16);
+    c.row = row;
+    c.m = m_tile * kBM + row;
+    c.n0 = n_tile * Cfg::BN;
+    c.split = split;
+    c.has_acc = nkb > 0;
+    Epi::template run<Cfg::BN>(ep, st, c, geom);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Cfg::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ epilogues
+
+__device__ __forceinline__ void store_bf16x8(__nv_bfloat16* dst, const float* v) {
+  __nv_bfloat162 p[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) p[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+  *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(p);
+}
+
+struct NoRowState {};
+
+// out[m, n] = alpha * acc  (or out[n, m] when transposed), bf16.
+struct EpiStoreBF16 {
+  struct Params {
+    __nv_bfloat16* out;
+    long long ldo;
+    float alpha;
+    int transpose;
+  };
+  using RowState = NoRowState;
+  static constexpr bool kReadsA = false;
+  __device__ static void on_a_stage(const Params&, RowState&, const uint8_t*, bool) {}
+  template <int BN>
+  __device__ static void run(const Params& p, RowState&, const EpiCtx& c, const GemmGeom& g) {
+    const bool row_ok = c.m < g.M;
+    for_each_acc_chunk<BN>(c, [&](int col, float* v) {
+      const int n = c.n0 + col;
+      if (!row_ok) return;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] *= p.alpha;
+      if (!p.transpose) {
+        __nv_bfloat16* dst = p.out + (long long)c.m * p.ldo + n;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (n + 8 * j < g.N) store_bf16x8(dst + 8 * j, v + 8 * j);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (n + i < g.N) p.out[(long long)(n + i) * p.ldo + c.m] = __float2bfloat16_rn(v[i]);
+      }
+    });
+  }
+};
+
+// part[split][m][n] = acc (fp32), row length ldp; summed later in split order.
+struct EpiPartialF32 {
+  struct Params {
+    float* part;
+    long long ldp;
+    long long split_stride;
+  };
+  using RowState = NoRowState;
+  static constexpr bool kReadsA = false;
+  __device__ static void on_a_stage(const Params&, RowState&, const uint8_t*, bool) {}
+  template <int BN>
+  __device__ static void run(const Params& p, RowState&, const EpiCtx& c, const GemmGeom& g) {
+    const bool row_ok = c.m < g.M;
+    float* base = p.part + (long long)c.split * p.split_stride + (long long)c.m * p.ldp;
+    for_each_acc_chunk<BN>(c, [&](int col, float* v) {
+      const int n = c.n0 + col;
+      if (!row_ok) return;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (n + 4 * j < g.N)
+          *reinterpret_cast<float4*>(base + n + 4 * j) = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    });
+  }
+};
+
+}  // namespace dora
