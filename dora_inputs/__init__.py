@@ -112,11 +112,13 @@ def _store(v64: np.ndarray, dtype: str) -> np.ndarray:
     raise ValueError(dtype)
 
 
-def make_inputs(wl: Workload, with_backward: bool = True) -> dict:
+def make_inputs(wl: Workload, with_backward: bool = True, token_seed: int | None = None) -> dict:
     """Draw one workload's tensors. Order of draws: W0, A, B, m factor, x, dy.
 
     Returns float32 numpy arrays (exact storage-precision values) plus 's' and,
-    for near-unity workloads, 'delta' with m = None.
+    for near-unity workloads, 'delta' with m = None. With token_seed, x and dy
+    come from their own stream (data-parallel ranks share the weights but not
+    the tokens).
     """
     rng = np.random.Generator(np.random.PCG64(wl.seed))
     w0_std = wl.w0_std if wl.w0_std is not None else 1.0 / math.sqrt(wl.d_in)
@@ -136,6 +138,8 @@ def make_inputs(wl: Workload, with_backward: bool = True) -> dict:
     else:
         out["delta"] = rng.uniform(-wl.delta, wl.delta, wl.d_out)
         out["m"] = None
+    if token_seed is not None:
+        rng = np.random.Generator(np.random.PCG64([wl.seed, token_seed]))
     out["x"] = _store(rng.standard_normal((wl.T, wl.d_in)) * x_std, wl.dtype)
     if with_backward:
         out["dy"] = _store(rng.standard_normal((wl.T, wl.d_out)), wl.dtype)

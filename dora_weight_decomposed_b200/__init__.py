@@ -20,7 +20,8 @@ import os
 import threading
 
 __all__ = ["DoraError", "load_library", "library_path", "dora_workspace_size", "dora_norm", "dora_forward",
-           "dora_backward", "dora_device_status", "dora_last_error", "dora_version", "DORA_OP_NORM",
+           "dora_backward", "dora_device_status", "dora_last_error", "dora_version", "dora_profile_start",
+           "dora_profile_stop", "dora_profile_count", "dora_profile_read", "DORA_OP_NORM",
            "DORA_OP_FORWARD", "DORA_OP_BACKWARD", "STATUS_NAMES", "EXPORTED_SYMBOLS"]
 
 DORA_BF16, DORA_FP32 = 0, 1
@@ -28,6 +29,7 @@ DORA_OP_NORM, DORA_OP_FORWARD, DORA_OP_BACKWARD = 0, 1, 2
 STATUS_NAMES = {0: "DORA_OK", 1: "DORA_EINVAL", 2: "DORA_EUNSUPPORTED", 3: "DORA_EWORKSPACE", 4: "DORA_ECUDA",
                 5: "DORA_ETIMEOUT"}
 EXPORTED_SYMBOLS = ("dora_workspace_size", "dora_norm", "dora_forward", "dora_backward", "dora_device_status",
+                    "dora_profile_start", "dora_profile_stop", "dora_profile_count", "dora_profile_read",
                     "dora_last_error", "dora_version")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -41,6 +43,10 @@ class DoraError(RuntimeError):
     def __init__(self, status: int, message: str):
         super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
         self.status = status
+
+
+class ProfileRecord(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char_p), ("ms", ctypes.c_float)]
 
 
 class DoraDesc(ctypes.Structure):
@@ -74,6 +80,14 @@ def load_library() -> ctypes.CDLL:
         lib.dora_backward.restype = ctypes.c_int
         lib.dora_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint)]
         lib.dora_device_status.restype = ctypes.c_int
+        lib.dora_profile_start.argtypes = [ctypes.c_int]
+        lib.dora_profile_start.restype = ctypes.c_int
+        lib.dora_profile_stop.argtypes = []
+        lib.dora_profile_stop.restype = ctypes.c_int
+        lib.dora_profile_count.argtypes = []
+        lib.dora_profile_count.restype = ctypes.c_int
+        lib.dora_profile_read.argtypes = [ctypes.POINTER(ProfileRecord), ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
+        lib.dora_profile_read.restype = ctypes.c_int
         lib.dora_last_error.argtypes = []
         lib.dora_last_error.restype = ctypes.c_char_p
         lib.dora_version.argtypes = []
@@ -231,3 +245,26 @@ def dora_device_status(stream=None) -> int:
     if st not in (0, 5):
         _check(st)
     return int(flags.value)
+
+
+def dora_profile_start(capacity: int = 4096) -> None:
+    """Time every kernel the library launches from now on (see include/dora.h)."""
+    _check(load_library().dora_profile_start(int(capacity)))
+
+
+def dora_profile_stop() -> None:
+    _check(load_library().dora_profile_stop())
+
+
+def dora_profile_count() -> int:
+    return int(load_library().dora_profile_count())
+
+
+def dora_profile_read() -> list[tuple[str, float]]:
+    """[(kernel name, milliseconds)] for the recorded launches, in launch order."""
+    lib = load_library()
+    n = lib.dora_profile_count()
+    recs = (ProfileRecord * max(n, 1))()
+    got = ctypes.c_int(0)
+    _check(lib.dora_profile_read(recs, n, ctypes.byref(got)))
+    return [(recs[i].name.decode(), float(recs[i].ms)) for i in range(got.value)]

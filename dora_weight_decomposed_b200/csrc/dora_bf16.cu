@@ -93,6 +93,7 @@ struct GemmArgs {
   int M = 0, N = 0;
   Split split;
   int a1_kwrap = 0;  // see GemmGeom::a1_kwrap
+  const char* name = "gemm";
 };
 
 // Raise the kernel's dynamic shared-memory limit once per device; `done` is
@@ -135,7 +136,10 @@ static cudaError_t launch_gemm(const GemmArgs& g, const typename Epi::Params& ep
     t_detail = "shared-memory attribute (" + std::to_string(Cfg::SMEM_BYTES) + " bytes)";
     return e;
   }
-  kern<<<grid, kGemmThreads, Cfg::SMEM_BYTES, st>>>(ta0, ta1, tb0, tb1, geom, ep);
+  {
+    ProfRange pr(g.name, st);
+    kern<<<grid, kGemmThreads, Cfg::SMEM_BYTES, st>>>(ta0, ta1, tb0, tb1, geom, ep);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess)
     t_detail = "launch grid (" + std::to_string(grid.x) + "," + std::to_string(grid.y) + "," +
@@ -432,6 +436,7 @@ static cudaError_t reduce_splits(const float* part, const Split& sp, long long s
   const long long total = (long long)M * (N / 4);
   const int threads = 256;
   const long long blocks = std::min<long long>(ceil_div(total, threads), 148LL * 16);
+  ProfRange pr("reduce_splits", st);
   reduce_splits_bf16_kernel<<<(unsigned)std::max<long long>(blocks, 1), threads, 0, st>>>(
       part, sp.splits, split_stride, M, N, alpha, out, ldo, transpose ? 1 : 0);
   return cudaGetLastError();
@@ -471,12 +476,14 @@ dora_status_t bf16_norm(const dora_desc_t& d, const Plan& p, const void* W0, con
   ga.M = r;
   ga.N = r;
   ga.split = p.gram;
+  ga.name = "gram_gemm";
   {
     const long long sstride = (long long)r * r;
     EpiPartialF32::Params pp{gram_part, r, sstride};
     cudaError_t e = gemm_bn<false, false, EpiPartialF32>(bn_skinny(r), ga, pp, st);
     if (e != cudaSuccess) return gemm_status(e, "dora_norm: Gram");
     const long long total = (long long)r * 2 * rp;
+    ProfRange pr("gram_finalize", st);
     gram_finalize_kernel<<<(unsigned)std::min<long long>(ceil_div(total, 256), 2048), 256, 0, st>>>(
         gram_part, p.gram.splits, r, rp, 0.5f * d.s, gs);
     e = cudaGetLastError();
@@ -495,12 +502,16 @@ dora_status_t bf16_norm(const dora_desc_t& d, const Plan& p, const void* W0, con
   na.M = d_out;
   na.N = r;
   na.split = p.norm;
+  na.name = "norm_gemm";
   EpiNorm::Params np{reinterpret_cast<const __nv_bfloat16*>(B), r, 2.0f * d.s, norm_part, d_out};
   cudaError_t e = norm_gemm(bn_norm(r), na, np, st);
   if (e != cudaSuccess) return gemm_status(e, "dora_norm: factored norm GEMM");
 
-  norm_finalize_kernel<<<(unsigned)ceil_div(d_out, 256), 256, 0, st>>>(norm_part, p.norm.splits, d_out, m, C, g,
-                                                                        gm1);
+  {
+    ProfRange pr("norm_finalize", st);
+    norm_finalize_kernel<<<(unsigned)ceil_div(d_out, 256), 256, 0, st>>>(norm_part, p.norm.splits, d_out, m, C, g,
+                                                                          gm1);
+  }
   return cuda_status(cudaGetLastError(), "dora_norm: finalize");
 }
 
@@ -520,6 +531,7 @@ dora_status_t bf16_forward(const dora_desc_t& d, const Plan& p, int64_t T, const
   ua.M = Ti;
   ua.N = r;
   ua.split = p.u;
+  ua.name = "u_gemm";
   cudaError_t e = narrow_gemm<false, false>(p.u_bn, ua, d.s, su, r, false,
                                             reinterpret_cast<float*>(ws + p.off_u_part), st);
   if (e != cudaSuccess) return gemm_status(e, "dora_forward: LoRA down projection");
@@ -535,6 +547,7 @@ dora_status_t bf16_forward(const dora_desc_t& d, const Plan& p, int64_t T, const
   ba.M = Ti;
   ba.N = d_out;
   ba.split.splits = 1;
+  ba.name = "fwd_compose_gemm";
   ba.split.kb_per_split = (int)(ceil_div(d_in, kBK) + ceil_div(r, kBK));
   EpiCompose::Params cp{reinterpret_cast<__nv_bfloat16*>(y), reinterpret_cast<__nv_bfloat16*>(pre_save), gm1,
                         d_out};
@@ -560,10 +573,16 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
   // dz = g * dy, dm = sum_t dy * pre / C
   {
     dim3 grid((unsigned)ceil_div(d_out, 64), (unsigned)p.dm_rowblocks);
-    compose_bwd_bf16_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(dy),
-                                                  reinterpret_cast<const __nv_bfloat16*>(pre), g, dz, dm_part,
-                                                  Ti, d_out);
-    dm_finalize_kernel<<<(unsigned)ceil_div(d_out, 256), 256, 0, st>>>(dm_part, p.dm_rowblocks, d_out, C, dm);
+    {
+      ProfRange pr("compose_bwd", st);
+      compose_bwd_bf16_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(dy),
+                                                    reinterpret_cast<const __nv_bfloat16*>(pre), g, dz, dm_part,
+                                                    Ti, d_out);
+    }
+    {
+      ProfRange pr("dm_finalize", st);
+      dm_finalize_kernel<<<(unsigned)ceil_div(d_out, 256), 256, 0, st>>>(dm_part, p.dm_rowblocks, d_out, C, dm);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_status(e, "dora_backward: compose backward");
   }
@@ -576,6 +595,7 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.M = Ti;
     a.N = r;
     a.split = p.du;
+    a.name = "du_gemm";
     cudaError_t e = narrow_gemm<false, true>(p.r_bn_mn, a, d.s, du, r, false,
                                              reinterpret_cast<float*>(ws + p.off_du_part), st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: du");
@@ -589,6 +609,7 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.M = d_out;
     a.N = r;
     a.split = p.dB;
+    a.name = "dB_gemm";
     cudaError_t e = narrow_gemm<true, true>(p.r_bn_mn, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dB), r, false,
                                             reinterpret_cast<float*>(ws + p.off_dB_part), st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: dB");
@@ -602,6 +623,7 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.M = d_in;
     a.N = r;
     a.split = p.dA;
+    a.name = "dA_gemm";
     cudaError_t e = narrow_gemm<true, true>(p.r_bn_mn, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dA), d_in, true,
                                             reinterpret_cast<float*>(ws + p.off_dA_part), st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: dA");
@@ -618,6 +640,7 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.M = Ti;
     a.N = d_in;
     a.split.splits = 1;
+    a.name = "dx_gemm";
     a.split.kb_per_split = (int)(ceil_div(d_out, kBK) + ceil_div(r, kBK));
     EpiStoreBF16::Params sp{reinterpret_cast<__nv_bfloat16*>(dx), d_in, 1.0f, 0};
     cudaError_t e = launch_gemm<GemmCfg<256, false, true>, EpiStoreBF16>(a, sp, st);

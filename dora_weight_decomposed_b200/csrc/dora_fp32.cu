@@ -72,6 +72,7 @@ static cudaError_t sgemm(int M, int N, int K, const float* A, long long sam, lon
                          cudaStream_t st) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   dim3 grid((unsigned)cdiv(N, 64), (unsigned)cdiv(M, 64));
+  ProfRange pr("sgemm", st);
   sgemm_strided_kernel<<<grid, 256, 0, st>>>(M, N, std::max(K, 0), A, sam, sak, B, sbn, sbk, C, ldc, alpha, beta);
   return cudaGetLastError();
 }
@@ -159,6 +160,7 @@ dora_status_t f32_norm(const dora_desc_t& d, const Plan& p, const float* W0, con
   if (e == cudaSuccess) e = sgemm(r, r, d_in, A, d_in, 1, A, d_in, 1, G, r, 1.f, 0.f, st);  // G = A A^T
   if (e == cudaSuccess) e = sgemm(d_out, r, r, B, r, 1, G, r, 1, Q, r, 1.f, 0.f, st);      // Q = B G
   if (e != cudaSuccess) return cuda_status(e, "dora_norm (fp32)");
+  ProfRange pr("f32_norm_rows", st);
   f32_norm_rows_kernel<<<(unsigned)cdiv(d_out, 8), 256, 0, st>>>(W0, B, P, Q, m, d_out, d_in, r, d.s, C, g, gm1);
   return cuda_status(cudaGetLastError(), "dora_norm (fp32)");
 }
@@ -175,6 +177,7 @@ dora_status_t f32_forward(const dora_desc_t& d, const Plan& p, int64_t T, const 
   if (e == cudaSuccess) e = sgemm(Ti, d_out, r, su, r, 1, B, r, 1, pre, d_out, 1.f, 1.f, st);          // + su B^T
   if (e != cudaSuccess) return cuda_status(e, "dora_forward (fp32)");
   const long long total = (long long)Ti * d_out;
+  ProfRange pr("f32_compose", st);
   f32_compose_kernel<<<(unsigned)std::min<long long>(cdiv(total, 256), 4096), 256, 0, st>>>(pre, gm1, y, total,
                                                                                             d_out);
   return cuda_status(cudaGetLastError(), "dora_forward (fp32)");
@@ -195,9 +198,15 @@ dora_status_t f32_backward(const dora_desc_t& d, const Plan& p, int64_t T, const
   float* part = reinterpret_cast<float*>(ws + p.off_f32_b);
   float* du = reinterpret_cast<float*>(ws + p.off_f32_c);
   const int rb = (int)cdiv(Ti, kF32Rows);
-  f32_compose_bwd_kernel<<<dim3((unsigned)cdiv(d_out, 128), (unsigned)rb), 128, 0, st>>>(dy, pre, g, dz, part, Ti,
-                                                                                         d_out);
-  f32_dm_finalize_kernel<<<(unsigned)cdiv(d_out, 256), 256, 0, st>>>(part, rb, d_out, C, dm);
+  {
+    ProfRange pr("f32_compose_bwd", st);
+    f32_compose_bwd_kernel<<<dim3((unsigned)cdiv(d_out, 128), (unsigned)rb), 128, 0, st>>>(dy, pre, g, dz, part,
+                                                                                           Ti, d_out);
+  }
+  {
+    ProfRange pr("f32_dm_finalize", st);
+    f32_dm_finalize_kernel<<<(unsigned)cdiv(d_out, 256), 256, 0, st>>>(part, rb, d_out, C, dm);
+  }
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) e = sgemm(Ti, r, d_out, dz, d_out, 1, B, 1, r, du, r, d.s, 0.f, st);      // du = s dz B
   if (e == cudaSuccess) e = sgemm(d_out, r, Ti, dz, 1, d_out, su, 1, r, dB, r, 1.f, 0.f, st);     // dB = dz^T su

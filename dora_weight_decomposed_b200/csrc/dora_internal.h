@@ -69,6 +69,19 @@ dora_status_t f32_backward(const dora_desc_t& d, const Plan& p, int64_t T, const
                            const float* su, const float* pre, float* dm, float* dA, float* dB, float* dx,
                            uint8_t* ws, cudaStream_t st);
 
+// Brackets one kernel launch with profiling events when profiling is on.
+class ProfRange {
+ public:
+  ProfRange(const char* name, cudaStream_t st);
+  ~ProfRange();
+  ProfRange(const ProfRange&) = delete;
+  ProfRange& operator=(const ProfRange&) = delete;
+
+ private:
+  cudaStream_t st_;
+  int idx_;
+};
+
 inline dora_status_t cuda_status(cudaError_t e, const char* where) {
   if (e == cudaSuccess) return DORA_OK;
   set_error(std::string(where) + ": " + cudaGetErrorString(e));

@@ -136,6 +136,25 @@ DORA_API dora_status_t dora_backward(const dora_desc_t* desc, int64_t T, const v
  */
 DORA_API dora_status_t dora_device_status(dora_stream_t stream, unsigned int* flags_out);
 
+/*
+ * Kernel timing (benchmarks and tracing; not part of the compute path).
+ * dora_profile_start(capacity) creates 2 * capacity CUDA events and, until
+ * dora_profile_stop(), brackets each kernel the library launches with a pair of
+ * them on the launch stream (as graph event-record nodes while the stream is
+ * captured, so every graph replay re-times the same kernels). dora_profile_read
+ * waits for the recorded events and fills up to `capacity` records in launch
+ * order; `name` points to a static string naming the kernel. One host thread.
+ */
+typedef struct {
+  const char* name;
+  float ms;
+} dora_profile_record_t;
+
+DORA_API dora_status_t dora_profile_start(int capacity);
+DORA_API dora_status_t dora_profile_stop(void);
+DORA_API int dora_profile_count(void);
+DORA_API dora_status_t dora_profile_read(dora_profile_record_t* out, int capacity, int* n_out);
+
 /* Message for the last non-OK status returned on this thread ("" if none). */
 DORA_API const char* dora_last_error(void);
 
