@@ -20,7 +20,8 @@ import os
 import threading
 
 __all__ = ["DoraError", "load_library", "library_path", "dora_workspace_size", "dora_norm", "dora_forward",
-           "dora_backward", "dora_device_status", "dora_last_error", "dora_version", "dora_profile_start",
+           "dora_norm_noalloc", "dora_backward", "dora_device_status", "dora_last_error", "dora_version",
+           "dora_profile_start",
            "dora_profile_stop", "dora_profile_count", "dora_profile_read", "DORA_OP_NORM",
            "DORA_OP_FORWARD", "DORA_OP_BACKWARD", "STATUS_NAMES", "EXPORTED_SYMBOLS"]
 
@@ -28,7 +29,8 @@ DORA_BF16, DORA_FP32 = 0, 1
 DORA_OP_NORM, DORA_OP_FORWARD, DORA_OP_BACKWARD = 0, 1, 2
 STATUS_NAMES = {0: "DORA_OK", 1: "DORA_EINVAL", 2: "DORA_EUNSUPPORTED", 3: "DORA_EWORKSPACE", 4: "DORA_ECUDA",
                 5: "DORA_ETIMEOUT"}
-EXPORTED_SYMBOLS = ("dora_workspace_size", "dora_norm", "dora_forward", "dora_backward", "dora_device_status",
+EXPORTED_SYMBOLS = ("dora_workspace_size", "dora_norm", "dora_norm_noalloc", "dora_forward", "dora_backward",
+                    "dora_device_status",
                     "dora_profile_start", "dora_profile_stop", "dora_profile_count", "dora_profile_read",
                     "dora_last_error", "dora_version")
 
@@ -268,3 +270,31 @@ def dora_profile_read() -> list[tuple[str, float]]:
     got = ctypes.c_int(0)
     _check(lib.dora_profile_read(recs, n, ctypes.byref(got)))
     return [(recs[i].name.decode(), float(recs[i].ms)) for i in range(got.value)]
+
+
+def dora_norm_noalloc(W0, A, B, m, s: float, *, norm_out=None, g_out=None, gm1_out=None, stream=None):
+    """dora_norm for callers that cannot allocate device memory for a workspace.
+
+    The library uses its own built-in 16 MiB device scratch array instead (see
+    include/dora.h); outputs may be passed in preallocated. Calls on one device
+    share that array, so calls that may overlap on the GPU must be ordered.
+    """
+    torch = _torch()
+    lib = load_library()
+    fn = lib.dora_norm_noalloc
+    P = ctypes.c_void_p
+    fn.argtypes = [ctypes.POINTER(DoraDesc), P, P, P, P, P, P, P, P]
+    fn.restype = ctypes.c_int
+    d_out, d_in = W0.shape
+    r = A.shape[0]
+    _shape(A, (r, d_in), "A")
+    _shape(B, (d_out, r), "B")
+    _shape(m, (d_out,), "m")
+    desc = _desc(d_out, d_in, r, W0.dtype, s)
+    f32 = dict(dtype=torch.float32, device=W0.device)
+    norm_out = torch.empty(d_out, **f32) if norm_out is None else norm_out
+    g_out = torch.empty(d_out, **f32) if g_out is None else g_out
+    gm1_out = torch.empty(d_out, **f32) if gm1_out is None else gm1_out
+    _check(fn(ctypes.byref(desc), _ptr(W0), _ptr(A), _ptr(B), _ptr(m), _ptr(norm_out), _ptr(g_out), _ptr(gm1_out),
+              _stream_ptr(stream)))
+    return norm_out, g_out, gm1_out

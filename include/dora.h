@@ -91,6 +91,28 @@ DORA_API dora_status_t dora_norm(const dora_desc_t* desc, const void* W0, const 
                         size_t ws_bytes, dora_stream_t stream);
 
 /*
+ * dora_norm_noalloc -- dora_norm without a workspace argument; it allocates nothing.
+ *
+ * The pages describe no such call; it exists for callers that cannot allocate
+ * device memory or hand over a workspace: applications whose memory manager
+ * already owns the device memory they may use, loops that must not trigger
+ * cudaMalloc's implicit synchronisation, and thin bindings that hold only the
+ * layer's tensors. Same inputs, outputs and results as dora_norm.
+ * Scratch: one 16 MiB (16,777,216-byte) device array inside the library, held
+ * by every GPU that loads it until the process exits. A layer whose norm needs
+ * more scratch than that (dora_workspace_size(desc, 0, DORA_OP_NORM) > 16 MiB)
+ * is rejected with DORA_EUNSUPPORTED before anything is launched.
+ * The first call on a device looks up the array's device address with that
+ * device current and caches it; make that first call before any stream
+ * capture. All calls on a device share the array and leave their contents in
+ * it (each call writes every scratch byte before reading it): calls whose
+ * kernels may overlap on the GPU race and must be ordered by the caller.
+ */
+DORA_API dora_status_t dora_norm_noalloc(const dora_desc_t* desc, const void* W0, const void* A, const void* B,
+                                         const float* m, float* norm_out, float* g_out, float* gm1_out,
+                                         dora_stream_t stream);
+
+/*
  * dora_forward -- y = x (diag(g) V')^T for T tokens, composed in one pass.
  *
  *   su  = s * x A^T                                   [T x r]
