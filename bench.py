@@ -50,7 +50,7 @@ def log(*a):
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description="DoRA layer step benchmark")
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD_KEY, help="workload key (c2, c3, c4a, c4b, c5)")
@@ -179,7 +179,8 @@ class ClockSampler:
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
                     "note": self.error or "no samples"}
-        loaded = [s for s in self.samples if s[2] > 0] or self.samples
+        # The sampler runs only inside the timed region, so every sample is under load.
+        loaded = self.samples
         bits = 0
         for _, rs, _ in loaded:
             bits |= rs

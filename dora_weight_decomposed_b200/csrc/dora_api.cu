@@ -26,20 +26,25 @@ int device_sm_count() {
 static inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 static inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-// Pick how many K splits a GEMM with `tiles` output tiles and `kb` k-blocks
-// gets: minimise (waves of one-CTA-per-SM) x (k-blocks per CTA + fixed cost).
-static Split choose_split(int64_t tiles, int64_t kb, int sms) {
+// Pick how many K splits a GEMM gets. Model (in units of one k-block's
+// main-loop time on one SM, kb_bytes of operands): each CTA costs its
+// k-blocks + 4 (prologue, TMEM, tails) + its output tile traffic (bf16 when
+// not split, fp32 partials when split); CTAs run in waves of one per SM; a
+// split GEMM adds a reduction pass over all partials (write + read).
+static Split choose_split(int64_t tiles, int64_t kb, int sms, double kb_bytes, double tile_out_elems,
+                          double out_elems, int64_t max_splits = 64) {
   Split best;
   best.splits = 1;
   best.kb_per_split = (int)std::max<int64_t>(kb, 1);
   if (kb <= 1 || tiles <= 0) return best;
-  const double fixed_cost = 4.0;
   double best_t = 1e300;
-  for (int64_t n = 1; n <= std::min<int64_t>(kb, 64); ++n) {
+  for (int64_t n = 1; n <= std::min<int64_t>(kb, std::max<int64_t>(max_splits, 1)); ++n) {
     const int64_t kps = cdiv(kb, n);
     const int64_t ns = cdiv(kb, kps);
     const int64_t waves = cdiv(tiles * ns, sms);
-    const double t = (double)waves * ((double)kps + fixed_cost);
+    const double tile_out = tile_out_elems * (ns > 1 ? 4.0 : 2.0) / kb_bytes;
+    const double reduce = ns > 1 ? (double)ns * out_elems * 8.0 / ((double)sms * kb_bytes) : 0.0;
+    const double t = (double)waves * ((double)kps + 4.0 + tile_out) + reduce;
     if (t < best_t - 1e-9) {
       best_t = t;
       best.splits = (int)ns;
@@ -48,8 +53,6 @@ static Split choose_split(int64_t tiles, int64_t kb, int sms) {
   }
   return best;
 }
-
-static int bn_skinny(int64_t r) { return r <= 16 ? 16 : r <= 32 ? 32 : r <= 64 ? 64 : 128; }
 
 Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
   Plan p;
@@ -62,30 +65,36 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
   };
   const int64_t r = d.r, d_in = d.d_in, d_out = d.d_out;
   if (d.dtype == DORA_BF16) {
+    const double kbB = 64.0 * 2.0;  // bytes per K element pair of rows (x 64 K per k-block)
     if (op == DORA_OP_NORM) {
-      const int64_t gram_tiles = cdiv(r, 128) * cdiv(r, bn_skinny(r));
-      p.gram = choose_split(gram_tiles, cdiv(d_in, 64), p.sms);
+      const int bk = bn_narrow_k(r);
+      // The Gram GEMM is small; its fp32 partials are capped at 8 MiB.
+      const int64_t gram_max = std::max<int64_t>(1, (int64_t(8) << 20) / (r * r * 4));
+      p.gram = choose_split(cdiv(r, 128), cdiv(d_in, 64), p.sms, kbB * (128 + bk), 128.0 * bk, (double)r * r,
+                            gram_max);
       p.off_gram_part = take((size_t)p.gram.splits * r * r * 4);
       p.off_gs = take((size_t)r * 2 * cdiv(r, 64) * 64 * 2);
-      p.norm = choose_split(cdiv(d_out, 128), cdiv(d_in, 64) + 2 * cdiv(r, 64), p.sms);
+      p.norm = choose_split(cdiv(d_out, 128), cdiv(d_in, 64) + 2 * cdiv(r, 64), p.sms, kbB * (128 + bk), 0.0,
+                            (double)d_out);
       p.off_norm_part = take((size_t)p.norm.splits * d_out * 4);
     } else if (op == DORA_OP_FORWARD && T > 0) {
-      p.u_bn = bn_skinny(r);
-      p.u = choose_split(cdiv(T, 128) * cdiv(r, p.u_bn), cdiv(d_in, 64), p.sms);
+      p.u_bn = bn_narrow_k(r);
+      p.u = choose_split(cdiv(T, 128), cdiv(d_in, 64), p.sms, kbB * (128 + p.u_bn), 128.0 * p.u_bn,
+                         (double)T * r);
       if (p.u.splits > 1) p.off_u_part = take((size_t)p.u.splits * T * r * 4);
       p.off_su = take((size_t)T * r * 2);
     } else if (op == DORA_OP_BACKWARD && T > 0) {
       p.off_dz = take((size_t)T * d_out * 2);
       p.dm_rowblocks = (int)cdiv(T, 256);
       p.off_dm_part = take((size_t)p.dm_rowblocks * d_out * 4);
-      p.r_bn_mn = r <= 64 ? 64 : 128;
-      const int64_t rnt = cdiv(r, p.r_bn_mn);
-      p.du = choose_split(cdiv(T, 128) * rnt, cdiv(d_out, 64), p.sms);
+      p.r_bn_mn = bn_narrow_mn(r);
+      const double kb_mn = kbB * (128 + p.r_bn_mn);
+      p.du = choose_split(cdiv(T, 128), cdiv(d_out, 64), p.sms, kb_mn, 128.0 * p.r_bn_mn, (double)T * r);
       if (p.du.splits > 1) p.off_du_part = take((size_t)p.du.splits * T * r * 4);
       p.off_du = take((size_t)T * r * 2);
-      p.dB = choose_split(cdiv(d_out, 128) * rnt, cdiv(T, 64), p.sms);
+      p.dB = choose_split(cdiv(d_out, 128), cdiv(T, 64), p.sms, kb_mn, 128.0 * p.r_bn_mn, (double)d_out * r);
       if (p.dB.splits > 1) p.off_dB_part = take((size_t)p.dB.splits * d_out * r * 4);
-      p.dA = choose_split(cdiv(d_in, 128) * rnt, cdiv(T, 64), p.sms);
+      p.dA = choose_split(cdiv(d_in, 128), cdiv(T, 64), p.sms, kb_mn, 128.0 * p.r_bn_mn, (double)d_in * r);
       if (p.dA.splits > 1) p.off_dA_part = take((size_t)p.dA.splits * d_in * r * 4);
     }
   } else {

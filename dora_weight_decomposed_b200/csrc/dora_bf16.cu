@@ -185,9 +185,6 @@ static cudaError_t launch_gemm_persistent(const GemmArgs& g, const typename Epi:
   return e;
 }
 
-// Tile width for the narrow (N = r) GEMMs with K-major B.
-static int bn_skinny(int64_t r) { return r <= 16 ? 16 : r <= 32 ? 32 : r <= 64 ? 64 : 128; }
-
 template <bool A_MN, bool B_MN, class Epi>
 static cudaError_t gemm_bn(int bn, const GemmArgs& g, const typename Epi::Params& ep, cudaStream_t st) {
   if constexpr (!B_MN) {
@@ -196,6 +193,9 @@ static cudaError_t gemm_bn(int bn, const GemmArgs& g, const typename Epi::Params
   }
   if (bn == 64) return launch_gemm<GemmCfg<64, A_MN, B_MN>, Epi>(g, ep, st);
   if (bn == 128) return launch_gemm<GemmCfg<128, A_MN, B_MN>, Epi>(g, ep, st);
+  if (bn == 256) return launch_gemm<GemmCfg<256, A_MN, B_MN>, Epi>(g, ep, st);
+  if (bn == 384) return launch_gemm<GemmCfg<384, A_MN, B_MN>, Epi>(g, ep, st);
+  if (bn == 512) return launch_gemm<GemmCfg<512, A_MN, B_MN>, Epi>(g, ep, st);
   return cudaErrorInvalidValue;
 }
 
@@ -226,34 +226,53 @@ struct EpiNorm {
     float ss = 0.f;
   };
   static constexpr bool kReadsA = true;
-  // row_ptr: this thread's 128-byte row of the W0 tile (swizzle only permutes
-  // 16-byte chunks inside the row, which a sum of squares does not see).
+  // row_ptr: this thread's 128-byte row of the swizzled W0 tile. The swizzle
+  // permutes the row's eight 16-byte chunks by (row mod 8), which a sum of
+  // squares does not see; reading chunk j ^ (row mod 8) at step j keeps the
+  // 32 lanes of a warp on distinct banks.
   __device__ static void on_a_stage(const Params&, RowState& st, const uint8_t* row_ptr, bool src1) {
     if (src1) return;
     const uint4* p = reinterpret_cast<const uint4*>(row_ptr);
+    const int t = (int)(smem_u32(row_ptr) >> 7) & 7;
     float acc = 0.f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       float f[8];
-      unpack_bf16x8(p[j], f);
+      unpack_bf16x8(p[j ^ t], f);
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc = fmaf(f[i], f[i], acc);
     }
     st.ss += acc;
   }
+  // The tile's B rows [128 x r] are brought into the (now idle) stage ring by
+  // TMA through the A source-1 map, in 64-column slabs of the same swizzled
+  // layout, then dotted with the accumulator rows.
   template <int BN>
   __device__ static void run(const Params& p, RowState& st, const EpiCtx& c, const GemmGeom& g) {
     const bool row_ok = c.m < g.M;
-    const __nv_bfloat16* brow = p.B + (long long)(row_ok ? c.m : 0) * p.r;
+    const int slabs = (p.r + 63) / 64;
+    const uint32_t bytes = (uint32_t)slabs * 16384u;
+    // All four epilogue warps are past their last stage reads before the refill.
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (c.row == 0) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive_expect_tx(c.aux_bar, bytes);
+      const int m0 = c.m - c.row;
+      for (int sl = 0; sl < slabs; ++sl) tma_load_2d(c.stage_smem + sl * 16384, c.tA1, c.aux_bar, sl * 64, m0);
+    }
+    mbar_wait(c.aux_bar, 0);
+    const int t = c.row & 7;
     float dot = 0.f;
     for_each_acc_chunk<BN>(c, [&](int col, float* v) {
-      if (!row_ok) return;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int n = col + 8 * j;
         if (n < p.r) {
+          const int slab = n >> 6, chunk = (n & 63) >> 3;
+          const uint4 w =
+              *reinterpret_cast<const uint4*>(c.stage_smem + slab * 16384 + c.row * 128 + ((chunk ^ t) << 4));
           float b[8];
-          unpack_bf16x8(*reinterpret_cast<const uint4*>(brow + n), b);
+          unpack_bf16x8(w, b);
 #pragma unroll
           for (int i = 0; i < 8; ++i) dot = fmaf(b[i], v[8 * j + i], dot);
         }
@@ -303,9 +322,6 @@ static cudaError_t norm_gemm_bn(const GemmArgs& g, const EpiNorm::Params& ep, cu
   return launch_gemm<GemmCfg<BN, false, false>, EpiNorm>(g, ep, st);
 }
 
-static int bn_norm(int64_t r) {
-  return r <= 16 ? 16 : r <= 32 ? 32 : r <= 64 ? 64 : r <= 128 ? 128 : r <= 256 ? 256 : r <= 384 ? 384 : 512;
-}
 
 static cudaError_t norm_gemm(int bn, const GemmArgs& g, const EpiNorm::Params& ep, cudaStream_t st) {
   switch (bn) {
@@ -518,7 +534,7 @@ dora_status_t bf16_norm(const dora_desc_t& d, const Plan& p, const void* W0, con
   {
     const long long sstride = (long long)r * r;
     EpiPartialF32::Params pp{gram_part, r, sstride};
-    cudaError_t e = gemm_bn<false, false, EpiPartialF32>(bn_skinny(r), ga, pp, st);
+    cudaError_t e = gemm_bn<false, false, EpiPartialF32>(bn_narrow_k(r), ga, pp, st);
     if (e != cudaSuccess) return gemm_status(e, "dora_norm: Gram");
     const long long total = (long long)r * 2 * rp;
     ProfRange pr("gram_finalize", st);
@@ -542,7 +558,7 @@ dora_status_t bf16_norm(const dora_desc_t& d, const Plan& p, const void* W0, con
   na.split = p.norm;
   na.name = "norm_gemm";
   EpiNorm::Params np{reinterpret_cast<const __nv_bfloat16*>(B), r, 2.0f * d.s, norm_part, d_out};
-  cudaError_t e = norm_gemm(bn_norm(r), na, np, st);
+  cudaError_t e = norm_gemm(bn_narrow_k(r), na, np, st);
   if (e != cudaSuccess) return gemm_status(e, "dora_norm: factored norm GEMM");
 
   {

@@ -38,6 +38,14 @@ struct Plan {
   size_t total = 0;
 };
 
+// Tile widths of the narrow (N = r) GEMMs: the whole rank in one N tile, so
+// the large operand is streamed once. K-major B tiles step in 16s up to 128,
+// then 256 / 384 / 512; MN-major B tiles are whole 64-column swizzle chunks.
+inline int bn_narrow_k(int64_t r) {
+  return r <= 16 ? 16 : r <= 32 ? 32 : r <= 64 ? 64 : r <= 128 ? 128 : r <= 256 ? 256 : r <= 384 ? 384 : 512;
+}
+inline int bn_narrow_mn(int64_t r) { return r <= 64 ? 64 : r <= 128 ? 128 : r <= 256 ? 256 : r <= 384 ? 384 : 512; }
+
 int device_sm_count();
 Plan make_plan(const dora_desc_t& d, int64_t T, int op);
 

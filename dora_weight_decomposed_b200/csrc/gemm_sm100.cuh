@@ -69,6 +69,12 @@ struct EpiCtx {
   int n0;          // first global output column of the tile
   int split;       // blockIdx.z
   bool has_acc;    // false when this split had no k-blocks (accumulator never written)
+  // Non-persistent kernel only: once the accumulator is complete the stage
+  // ring is idle, and an epilogue may refill it through its own barrier.
+  uint8_t* stage_smem;        // start of the stage ring
+  int stage_bytes;            // bytes of the ring
+  uint64_t* aux_bar;          // spare mbarrier (count 1), phase 0 unused so far
+  const CUtensorMap* tA1;     // A-operand source-1 tensor map
 };
 
 // 16-column TMEM load (for tiles whose width is an odd multiple of 16).
@@ -124,7 +130,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* accf = empty + STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  uint64_t* aux = accf + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aux + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -143,6 +150,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&empty[s], 1 + (Epi::kReadsA ? 4 : 0));
     }
     mbar_init(accf, 1);
+    mbar_init(aux, 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -258,6 +266,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     c.n0 = n_tile * Cfg::BN;
     c.split = split;
     c.has_acc = nkb > 0;
+    c.stage_smem = smem;
+    c.stage_bytes = STAGES * Cfg::STAGE_BYTES;
+    c.aux_bar = aux;
+    c.tA1 = &tA1;
     Epi::template run<Cfg::BN>(ep, st, c, geom);
   }
 
@@ -443,6 +455,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       c.n0 = n_tile * Cfg::BN;
       c.split = 0;
       c.has_acc = nkb > 0;
+      c.stage_smem = nullptr;
+      c.stage_bytes = 0;
+      c.aux_bar = nullptr;
+      c.tA1 = &tA1;
       Epi::template run<Cfg::BN>(ep, st, c, geom);
       tc_fence_before();
       __syncwarp();
