@@ -185,6 +185,43 @@ static cudaError_t launch_gemm_persistent(const GemmArgs& g, const typename Epi:
   return e;
 }
 
+// CTA-pair persistent launch: clusters of two CTAs, one pair per two SMs.
+template <class Cfg, class Epi>
+static cudaError_t launch_gemm_pair(const GemmArgs& g, const typename Epi::Params& ep, int sms, cudaStream_t st) {
+  CUtensorMap ta0, ta1, tb0, tb1;
+  const int a_box = Cfg::A_MN ? 64 : kBM;
+  const int b_box = Cfg::B_MN ? 64 : Cfg::B_BOX;
+  t_detail.clear();
+  if (!make_map(&ta0, g.a0, a_box, "A source 0") || !make_map(&tb0, g.b0, b_box, "B source 0"))
+    return cudaErrorInvalidValue;
+  const int kb0 = (int)ceil_div(g.K0, kBK);
+  const int kb1 = g.K1 > 0 ? (int)ceil_div(g.K1, kBK) : 0;
+  if (kb1 > 0) {
+    if (!make_map(&ta1, g.a1, a_box, "A source 1") || !make_map(&tb1, g.b1, b_box, "B source 1"))
+      return cudaErrorInvalidValue;
+  } else {
+    ta1 = ta0;
+    tb1 = tb0;
+  }
+  GemmGeom geom{g.M, g.N, kb0, kb1, kb0 + kb1, g.a1_kwrap};
+  const long long tiles = ceil_div(g.N, Cfg::BN) * ceil_div(g.M, 2 * kBM);
+  const long long pairs = std::max<long long>(1, std::min<long long>(tiles, sms / 2));
+  auto kern = gemm_sm100_pair_kernel<Cfg, Epi>;
+  static std::atomic<unsigned long long> smem_set{0};
+  cudaError_t e = set_smem_once(smem_set, kern, Cfg::SMEM_BYTES);
+  if (e != cudaSuccess) {
+    t_detail = "shared-memory attribute (" + std::to_string(Cfg::SMEM_BYTES) + " bytes)";
+    return e;
+  }
+  {
+    ProfRange pr(g.name, st);
+    kern<<<(unsigned)(2 * pairs), kGemmThreads, Cfg::SMEM_BYTES, st>>>(ta0, ta1, tb0, tb1, geom, ep);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) t_detail = "pair launch, " + std::to_string(pairs) + " clusters of 2";
+  return e;
+}
+
 template <bool A_MN, bool B_MN, class Epi>
 static cudaError_t gemm_bn(int bn, const GemmArgs& g, const typename Epi::Params& ep, cudaStream_t st) {
   if constexpr (!B_MN) {
@@ -605,7 +642,7 @@ dora_status_t bf16_forward(const dora_desc_t& d, const Plan& p, int64_t T, const
   ba.split.kb_per_split = (int)(ceil_div(d_in, kBK) + ceil_div(r, kBK));
   EpiCompose::Params cp{reinterpret_cast<__nv_bfloat16*>(y), reinterpret_cast<__nv_bfloat16*>(pre_save), gm1,
                         d_out};
-  e = launch_gemm_persistent<GemmCfg<256, false, false>, EpiCompose>(ba, cp, p.sms, st);
+  e = launch_gemm_pair<PairCfg<256, false, false>, EpiCompose>(ba, cp, p.sms, st);
   return gemm_status(e, "dora_forward: base GEMM with compose");
 }
 
@@ -697,7 +734,7 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.name = "dx_gemm";
     a.split.kb_per_split = (int)(ceil_div(d_out, kBK) + ceil_div(r, kBK));
     EpiStoreBF16::Params sp{reinterpret_cast<__nv_bfloat16*>(dx), d_in, 1.0f, 0};
-    cudaError_t e = launch_gemm_persistent<GemmCfg<256, false, true>, EpiStoreBF16>(a, sp, p.sms, st);
+    cudaError_t e = launch_gemm_pair<PairCfg<256, false, true>, EpiStoreBF16>(a, sp, p.sms, st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: dx");
   }
   return DORA_OK;

@@ -474,6 +474,213 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ CTA-pair persistent variant
+//
+// A cluster of two CTAs computes 256 x BN output tiles with tcgen05.mma
+// cta_group::2: each CTA stages its own 128 rows of A and half of the B tile
+// (BN/2 rows), so per-SM operand traffic and shared memory per stage drop and
+// the ring gets deeper. Both CTAs' TMA loads complete on the leader CTA's
+// full barrier; the leader issues the MMAs and commits to the empty and
+// accumulator barriers of both CTAs; each CTA's epilogue drains its own TMEM
+// rows and reports to the leader. Tiles are walked persistently as above.
+template <int BN_, bool A_MN_, bool B_MN_>
+struct PairCfg {
+  static constexpr int BN = BN_;
+  static constexpr bool A_MN = A_MN_;
+  static constexpr bool B_MN = B_MN_;
+  static constexpr int BH = BN / 2;  // B rows (N) staged by each CTA
+  static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "pair tile N");
+  static_assert(!B_MN || BH % 64 == 0, "MN-major B halves are whole 64-wide chunks");
+  static constexpr int A_BYTES = kBM * kBK * 2;
+  static constexpr int B_BYTES = BH * kBK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES_RAW = kSmemBudget / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+  static constexpr int B_BOX = B_MN ? 64 : (BH <= 128 ? BH : 128);
+  static constexpr int B_LOADS = BH / B_BOX;
+  static constexpr uint32_t ACC_COLS = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
+};
+
+template <class Cfg, class Epi>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_sm100_pair_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tA1,
+                           const __grid_constant__ CUtensorMap tB0, const __grid_constant__ CUtensorMap tB1,
+                           const GemmGeom geom, const typename Epi::Params ep) {
+  static_assert(!Epi::kReadsA, "pair epilogues do not read A stages");
+  constexpr int STAGES = Cfg::STAGES;
+  constexpr uint32_t ACC_COLS = Cfg::ACC_COLS;
+  constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accf = empty + STAGES;  // [2]
+  uint64_t* acce = accf + 2;        // [2], used in the leader only
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+  const int m_tiles = (geom.M + 2 * kBM - 1) / (2 * kBM);
+  const int n_tiles = (geom.N + Cfg::BN - 1) / Cfg::BN;
+  const int tiles = m_tiles * n_tiles;
+  const int nkb = geom.kb0 + geom.kb1;
+
+  if (threadIdx.x == 0) {
+#pragma unroll 1
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accf[b], 1);
+      mbar_init(&acce[b], 8);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tA0);
+    prefetch_tmap(&tB0);
+    if (geom.kb1 > 0) {
+      prefetch_tmap(&tA1);
+      prefetch_tmap(&tB1);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+#pragma unroll 1
+      for (int t = pair; t < tiles && ok; t += npairs) {
+        int tm, tn;
+        tile_coords(t, m_tiles, n_tiles, tm, tn);
+        const int m0 = tm * 2 * kBM + (int)rank * kBM;
+        const int nb = tn * Cfg::BN + (int)rank * Cfg::BH;
+#pragma unroll 1
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + s * Cfg::STAGE_BYTES;
+          uint8_t* sb = sa + Cfg::A_BYTES;
+          const uint32_t fb = mapa_shared(smem_u32(&full[s]), 0);
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
+          const bool src1 = kb >= geom.kb0;
+          const int k0 = (src1 ? kb - geom.kb0 : kb) * kBK;
+          const int k0a = (src1 && geom.a1_kwrap > 0) ? k0 % geom.a1_kwrap : k0;
+          const CUtensorMap* ta = src1 ? &tA1 : &tA0;
+          const CUtensorMap* tb = src1 ? &tB1 : &tB0;
+          if (!Cfg::A_MN) {
+            tma_load_2d_pair(sa, ta, fb, k0a, m0);
+          } else {
+            tma_load_2d_pair(sa, ta, fb, m0, k0a);
+            tma_load_2d_pair(sa + 8192, ta, fb, m0 + 64, k0a);
+          }
+#pragma unroll
+          for (int j = 0; j < Cfg::B_LOADS; ++j) {
+            if (!Cfg::B_MN)
+              tma_load_2d_pair(sb + j * Cfg::B_BOX * 128, tb, fb, k0, nb + j * Cfg::B_BOX);
+            else
+              tma_load_2d_pair(sb + j * 8192, tb, fb, nb + j * 64, k0);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(2 * kBM, Cfg::BN, Cfg::A_MN, Cfg::B_MN);
+      constexpr uint32_t a_kstep = Cfg::A_MN ? 2048u : 32u;
+      constexpr uint32_t b_kstep = Cfg::B_MN ? 2048u : 32u;
+      constexpr uint32_t a_lbo = Cfg::A_MN ? 8192u : 16u;
+      constexpr uint32_t b_lbo = Cfg::B_MN ? 8192u : 16u;
+      int it = 0, j = 0;
+      bool ok = true;
+#pragma unroll 1
+      for (int t = pair; t < tiles && ok; t += npairs, ++j) {
+        const int b = j & 1;
+        const uint32_t uph = (uint32_t)(j >> 1) & 1u;
+        if (!mbar_wait(&acce[b], uph ^ 1u)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)b * ACC_COLS;
+#pragma unroll 1
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!mbar_wait(&full[s], ph)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * Cfg::STAGE_BYTES);
+          const uint32_t sb = sa + Cfg::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(sa + kk * a_kstep, a_lbo, 1024u);
+            const uint64_t bd = sdesc_sw128(sb + kk * b_kstep, b_lbo, 1024u);
+            umma_bf16_pair(d_tmem, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit_pair(&empty[s], 0x3);
+        }
+        umma_commit_pair(&accf[b], 0x3);
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    typename Epi::RowState st{};
+    int j = 0;
+#pragma unroll 1
+    for (int t = pair; t < tiles; t += npairs, ++j) {
+      const int b = j & 1;
+      const uint32_t uph = (uint32_t)(j >> 1) & 1u;
+      if (!mbar_wait(&accf[b], uph)) break;
+      tc_fence_after();
+      int tm, tn;
+      tile_coords(t, m_tiles, n_tiles, tm, tn);
+      EpiCtx c;
+      c.taddr = tmem + (uint32_t)b * ACC_COLS + ((uint32_t)(q * 32) << 16);
+      c.row = row;
+      c.m = tm * 2 * kBM + (int)rank * kBM + row;
+      c.n0 = tn * Cfg::BN;
+      c.split = 0;
+      c.has_acc = nkb > 0;
+      c.stage_smem = nullptr;
+      c.stage_bytes = 0;
+      c.aux_bar = nullptr;
+      c.tA1 = &tA1;
+      Epi::template run<Cfg::BN>(ep, st, c, geom);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acce[b]), 0));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ epilogues
 
 __device__ __forceinline__ void store_bf16x8(__nv_bfloat16* dst, const float* v) {
