@@ -73,10 +73,14 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
       p.gram = choose_split(cdiv(r, 128), cdiv(d_in, 64), p.sms, kbB * (128 + bk), 128.0 * bk, (double)r * r,
                             gram_max);
       p.off_gram_part = take((size_t)p.gram.splits * r * r * 4);
-      p.off_gs = take((size_t)r * 2 * cdiv(r, 64) * 64 * 2);
       p.norm = choose_split(cdiv(d_out, 128), cdiv(d_in, 64) + 2 * cdiv(r, 64), p.sms, kbB * (128 + bk), 0.0,
                             (double)d_out);
       p.off_norm_part = take((size_t)p.norm.splits * d_out * 4);
+      p.off_gs = take((size_t)r * 2 * cdiv(r, 64) * 64 * 2);
+      // split counters of the norm's row tiles, zeroed by one memset per call
+      p.gram_tiles = 0;
+      p.zero_bytes = (size_t)cdiv(d_out, 128) * 4;
+      p.off_ctr = take(p.zero_bytes);
     } else if (op == DORA_OP_FORWARD && T > 0) {
       p.u_bn = bn_narrow_k(r);
       p.u = choose_split(cdiv(T, 128), cdiv(d_in, 64), p.sms, kbB * (128 + p.u_bn), 128.0 * p.u_bn,
@@ -96,6 +100,9 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
       if (p.dB.splits > 1) p.off_dB_part = take((size_t)p.dB.splits * d_out * r * 4);
       p.dA = choose_split(cdiv(d_in, 128), cdiv(T, 64), p.sms, kb_mn, 128.0 * p.r_bn_mn, (double)d_in * r);
       if (p.dA.splits > 1) p.off_dA_part = take((size_t)p.dA.splits * d_in * r * 4);
+      // counters of the dm column strips, zeroed by one memset per call
+      p.zero_bytes = (size_t)cdiv(d_out, 64) * 4;
+      p.off_ctr = take(p.zero_bytes);
     }
   } else {
     if (op == DORA_OP_NORM) {

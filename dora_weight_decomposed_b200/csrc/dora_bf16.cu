@@ -258,10 +258,23 @@ struct EpiNorm {
     float two_s;
     float* part;             // [splits][d_out]
     int d_out;
+    unsigned int* counters;  // one per 128-row tile, zero before the launch
+    const float* m;          // magnitude [d_out]
+    float* C;                // outputs [d_out]
+    float* g;
+    float* gm1;
   };
   struct RowState {
     float ss = 0.f;
   };
+  // C = sqrt(max(0, sum of squares)), g = m / C, g - 1 = (m - C) / C.
+  __device__ static void finish(const Params& p, int m, float sq) {
+    const float c = sqrtf(fmaxf(sq, 0.f));
+    const float mi = p.m[m];
+    p.C[m] = c;
+    p.g[m] = mi / c;
+    p.gm1[m] = (mi - c) / c;
+  }
   static constexpr bool kReadsA = true;
   // row_ptr: this thread's 128-byte row of the swizzled W0 tile. The swizzle
   // permutes the row's eight 16-byte chunks by (row mod 8), which a sum of
@@ -315,9 +328,19 @@ struct EpiNorm {
         }
       }
     });
-    if (row_ok) p.part[(long long)c.split * p.d_out + c.m] = fmaf(p.two_s, dot, st.ss);
+    const float part = fmaf(p.two_s, dot, st.ss);
+    if (c.splits == 1) {
+      if (row_ok) finish(p, c.m, part);
+      return;
+    }
+    if (row_ok) p.part[(long long)c.split * p.d_out + c.m] = part;
+    if (!split_arrive_last(c, p.counters) || !row_ok) return;
+    float sq = 0.f;
+    for (int z = 0; z < c.splits; ++z) sq += __ldcg(p.part + (long long)z * p.d_out + c.m);
+    finish(p, c.m, sq);
   }
 };
+
 
 // Near-unity compose: y = pre + gm1[n] * pre (fp32, rounded once), pre optional.
 struct EpiCompose {
@@ -434,36 +457,27 @@ __global__ void gram_finalize_kernel(const float* __restrict__ part, int splits,
   }
 }
 
-// C = sqrt(max(0, sum of partials)), g = m / C, gm1 = (m - C) / C.
-__global__ void norm_finalize_kernel(const float* __restrict__ part, int nparts, int d_out,
-                                     const float* __restrict__ m, float* __restrict__ C, float* __restrict__ g,
-                                     float* __restrict__ gm1) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= d_out) return;
-  float sq = 0.f;
-  for (int z = 0; z < nparts; ++z) sq += part[(long long)z * d_out + i];
-  const float c = sqrtf(fmaxf(sq, 0.f));
-  const float mi = m[i];
-  C[i] = c;
-  g[i] = mi / c;
-  gm1[i] = (mi - c) / c;
-}
-
 // Compose backward, one streaming pass over [T x d_out]:
 //   dz[t][i] = g_i * dy[t][i]   (bf16)
 //   part[rb][i] = sum over the row block's t of dy[t][i] * pre[t][i]
 // Block: 256 threads, 64 columns x kCbRows rows. Lane = (row offset 0..3,
 // 8-column vector 0..7), so each warp access covers 4 full 128-byte rows; the
 // per-column sums are combined over the 4 row lanes with shuffles, then over
-// the 8 warps in shared memory.
+// the 8 warps in shared memory. The last row block of a column strip to
+// finish (counter per strip, zero before the launch) sums the strip's
+// partials in row-block order: dm_i = sum / C_i.
 constexpr int kCbRows = 256;
 
 __global__ void __launch_bounds__(256) compose_bwd_bf16_kernel(const __nv_bfloat16* __restrict__ dy,
                                                                const __nv_bfloat16* __restrict__ pre,
                                                                const float* __restrict__ g,
+                                                               const float* __restrict__ C,
                                                                __nv_bfloat16* __restrict__ dz,
-                                                               float* __restrict__ part, int T, int d_out) {
+                                                               float* __restrict__ part,
+                                                               unsigned int* __restrict__ counters,
+                                                               float* __restrict__ dm, int T, int d_out) {
   __shared__ float red[8][64];
+  __shared__ unsigned int last_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cv = lane & 7, ro = lane >> 3;
   const int col = blockIdx.x * 64 + cv * 8;
@@ -503,31 +517,32 @@ __global__ void __launch_bounds__(256) compose_bwd_bf16_kernel(const __nv_bfloat
     for (int j = 0; j < 8; ++j) red[warp][cv * 8 + j] = acc[j];
   }
   __syncthreads();
+  const int c = blockIdx.x * 64 + (int)threadIdx.x;
   if (threadIdx.x < 64) {
     float s = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) s += red[w][threadIdx.x];
-    const int c = blockIdx.x * 64 + threadIdx.x;
     if (c < d_out) part[(size_t)blockIdx.y * d_out + c] = s;
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last_flag = (atomicAdd(&counters[blockIdx.x], 1u) == gridDim.y - 1) ? 1u : 0u;
+  __syncthreads();
+  if (last_flag && threadIdx.x < 64 && c < d_out) {
+    __threadfence();
+    float s = 0.f;
+    for (unsigned int rb = 0; rb < gridDim.y; ++rb) s += __ldcg(part + (size_t)rb * d_out + c);
+    dm[c] = s / C[c];
   }
 }
 
-// dm_i = (sum over row blocks of part[rb][i]) / C_i.
-__global__ void dm_finalize_kernel(const float* __restrict__ part, int nparts, int d_out,
-                                   const float* __restrict__ C, float* __restrict__ dm) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= d_out) return;
-  float s = 0.f;
-  for (int z = 0; z < nparts; ++z) s += part[(long long)z * d_out + i];
-  dm[i] = s / C[i];
-}
-
 static cudaError_t reduce_splits(const float* part, const Split& sp, long long split_stride, int M, int N,
-                                 float alpha, __nv_bfloat16* out, long long ldo, bool transpose, cudaStream_t st) {
+                                 float alpha, __nv_bfloat16* out, long long ldo, bool transpose, const char* name,
+                                 cudaStream_t st) {
   const long long total = (long long)M * (N / 4);
   const int threads = 256;
   const long long blocks = std::min<long long>(ceil_div(total, threads), 148LL * 16);
-  ProfRange pr("reduce_splits", st);
+  ProfRange pr(name, st);
   reduce_splits_bf16_kernel<<<(unsigned)std::max<long long>(blocks, 1), threads, 0, st>>>(
       part, sp.splits, split_stride, M, N, alpha, out, ldo, transpose ? 1 : 0);
   return cudaGetLastError();
@@ -537,7 +552,7 @@ static cudaError_t reduce_splits(const float* part, const Split& sp, long long s
 // K loop is not split, else fp32 partials summed by reduce_splits.
 template <bool A_MN, bool B_MN>
 static cudaError_t narrow_gemm(int bn, const GemmArgs& g, float alpha, __nv_bfloat16* out, long long ldo,
-                               bool transpose, float* part, cudaStream_t st) {
+                               bool transpose, float* part, const char* reduce_name, cudaStream_t st) {
   if (g.split.splits == 1) {
     EpiStoreBF16::Params p{out, ldo, alpha, transpose ? 1 : 0};
     return gemm_bn<A_MN, B_MN, EpiStoreBF16>(bn, g, p, st);
@@ -546,7 +561,7 @@ static cudaError_t narrow_gemm(int bn, const GemmArgs& g, float alpha, __nv_bflo
   EpiPartialF32::Params p{part, g.N, sstride};
   cudaError_t e = gemm_bn<A_MN, B_MN, EpiPartialF32>(bn, g, p, st);
   if (e != cudaSuccess) return e;
-  return reduce_splits(part, g.split, sstride, g.M, g.N, alpha, out, ldo, transpose, st);
+  return reduce_splits(part, g.split, sstride, g.M, g.N, alpha, out, ldo, transpose, reduce_name, st);
 }
 
 // ============================================================== operations
@@ -557,6 +572,10 @@ dora_status_t bf16_norm(const dora_desc_t& d, const Plan& p, const void* W0, con
   float* gram_part = reinterpret_cast<float*>(ws + p.off_gram_part);
   __nv_bfloat16* gs = reinterpret_cast<__nv_bfloat16*>(ws + p.off_gs);
   float* norm_part = reinterpret_cast<float*>(ws + p.off_norm_part);
+  unsigned int* ctr = reinterpret_cast<unsigned int*>(ws + p.off_ctr);
+  // The norm's split counters start at zero.
+  cudaError_t e = cudaMemsetAsync(ws + p.off_ctr, 0, p.zero_bytes, st);
+  if (e != cudaSuccess) return cuda_status(e, "dora_norm: clearing counters");
 
   // Gram G = A A^T in fp32 partials, then (s/2) G as bf16 hi and lo halves.
   const int rp = (int)ceil_div(r, kBK) * kBK;
@@ -571,7 +590,7 @@ dora_status_t bf16_norm(const dora_desc_t& d, const Plan& p, const void* W0, con
   {
     const long long sstride = (long long)r * r;
     EpiPartialF32::Params pp{gram_part, r, sstride};
-    cudaError_t e = gemm_bn<false, false, EpiPartialF32>(bn_narrow_k(r), ga, pp, st);
+    e = gemm_bn<false, false, EpiPartialF32>(bn_narrow_k(r), ga, pp, st);
     if (e != cudaSuccess) return gemm_status(e, "dora_norm: Gram");
     const long long total = (long long)r * 2 * rp;
     ProfRange pr("gram_finalize", st);
@@ -581,7 +600,8 @@ dora_status_t bf16_norm(const dora_desc_t& d, const Plan& p, const void* W0, con
     if (e != cudaSuccess) return cuda_status(e, "dora_norm: Gram finalize");
   }
 
-  // acc = [W0 | B | B] [A | Gs_hi | Gs_lo]^T with the factored-norm epilogue.
+  // acc = [W0 | B | B] [A | Gs_hi | Gs_lo]^T with the factored-norm epilogue,
+  // finished (C, g, g - 1) by the last split of each row tile.
   GemmArgs na;
   na.a0 = Mat{W0, d_out, d_in, d_in};
   na.a1 = Mat{B, d_out, r, r};
@@ -594,16 +614,10 @@ dora_status_t bf16_norm(const dora_desc_t& d, const Plan& p, const void* W0, con
   na.N = r;
   na.split = p.norm;
   na.name = "norm_gemm";
-  EpiNorm::Params np{reinterpret_cast<const __nv_bfloat16*>(B), r, 2.0f * d.s, norm_part, d_out};
-  cudaError_t e = norm_gemm(bn_narrow_k(r), na, np, st);
-  if (e != cudaSuccess) return gemm_status(e, "dora_norm: factored norm GEMM");
-
-  {
-    ProfRange pr("norm_finalize", st);
-    norm_finalize_kernel<<<(unsigned)ceil_div(d_out, 256), 256, 0, st>>>(norm_part, p.norm.splits, d_out, m, C, g,
-                                                                          gm1);
-  }
-  return cuda_status(cudaGetLastError(), "dora_norm: finalize");
+  EpiNorm::Params np{reinterpret_cast<const __nv_bfloat16*>(B), r, 2.0f * d.s, norm_part, d_out,
+                     ctr + p.gram_tiles, m, C, g, gm1};
+  e = norm_gemm(bn_narrow_k(r), na, np, st);
+  return gemm_status(e, "dora_norm: factored norm GEMM");
 }
 
 dora_status_t bf16_forward(const dora_desc_t& d, const Plan& p, int64_t T, const void* x, const void* W0,
@@ -623,8 +637,8 @@ dora_status_t bf16_forward(const dora_desc_t& d, const Plan& p, int64_t T, const
   ua.N = r;
   ua.split = p.u;
   ua.name = "u_gemm";
-  cudaError_t e = narrow_gemm<false, false>(p.u_bn, ua, d.s, su, r, false,
-                                            reinterpret_cast<float*>(ws + p.off_u_part), st);
+  cudaError_t e = narrow_gemm<false, false>(p.u_bn, ua, d.s, su, r, false, reinterpret_cast<float*>(ws + p.off_u_part),
+                                "u_reduce", st);
   if (e != cudaSuccess) return gemm_status(e, "dora_forward: LoRA down projection");
 
   // pre = [x | su] [W0 | B]^T, y = pre + gm1 * pre
@@ -661,18 +675,20 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
   float* dm_part = reinterpret_cast<float*>(ws + p.off_dm_part);
   __nv_bfloat16* du = reinterpret_cast<__nv_bfloat16*>(ws + p.off_du);
 
+  unsigned int* ctr = reinterpret_cast<unsigned int*>(ws + p.off_ctr);
+  {
+    cudaError_t e = cudaMemsetAsync(ws + p.off_ctr, 0, p.zero_bytes, st);
+    if (e != cudaSuccess) return cuda_status(e, "dora_backward: clearing counters");
+  }
   // dz = g * dy, dm = sum_t dy * pre / C
   {
-    dim3 grid((unsigned)ceil_div(d_out, 64), (unsigned)p.dm_rowblocks);
+    const unsigned col_tiles = (unsigned)ceil_div(d_out, 64);
+    dim3 grid(col_tiles, (unsigned)p.dm_rowblocks);
     {
       ProfRange pr("compose_bwd", st);
       compose_bwd_bf16_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(dy),
-                                                    reinterpret_cast<const __nv_bfloat16*>(pre), g, dz, dm_part,
-                                                    Ti, d_out);
-    }
-    {
-      ProfRange pr("dm_finalize", st);
-      dm_finalize_kernel<<<(unsigned)ceil_div(d_out, 256), 256, 0, st>>>(dm_part, p.dm_rowblocks, d_out, C, dm);
+                                                    reinterpret_cast<const __nv_bfloat16*>(pre), g, C, dz, dm_part,
+                                                    ctr, dm, Ti, d_out);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_status(e, "dora_backward: compose backward");
@@ -688,7 +704,7 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.split = p.du;
     a.name = "du_gemm";
     cudaError_t e = narrow_gemm<false, true>(p.r_bn_mn, a, d.s, du, r, false,
-                                             reinterpret_cast<float*>(ws + p.off_du_part), st);
+                                             reinterpret_cast<float*>(ws + p.off_du_part), "du_reduce", st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: du");
   }
   // dB = dz^T su  (both token-major: K = T)
@@ -702,7 +718,7 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.split = p.dB;
     a.name = "dB_gemm";
     cudaError_t e = narrow_gemm<true, true>(p.r_bn_mn, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dB), r, false,
-                                            reinterpret_cast<float*>(ws + p.off_dB_part), st);
+                                            reinterpret_cast<float*>(ws + p.off_dB_part), "dB_reduce", st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: dB");
   }
   // dA^T = x^T du, stored transposed into dA [r x d_in]
@@ -716,7 +732,7 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.split = p.dA;
     a.name = "dA_gemm";
     cudaError_t e = narrow_gemm<true, true>(p.r_bn_mn, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dA), d_in, true,
-                                            reinterpret_cast<float*>(ws + p.off_dA_part), st);
+                                            reinterpret_cast<float*>(ws + p.off_dA_part), "dA_reduce", st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: dA");
   }
   // dx = [dz | du] [W0 ; A]  (W0 and A read MN-major: K rows, N = d_in contiguous)

@@ -33,6 +33,9 @@ struct Plan {
   Split du, dB, dA;
   int r_bn_mn = 0;
   size_t off_dz = 0, off_dm_part = 0, off_du_part = 0, off_du = 0, off_dB_part = 0, off_dA_part = 0;
+  // split counters (+ padding that must start at zero), cleared by one memset per call
+  size_t off_ctr = 0, zero_bytes = 0;
+  int gram_tiles = 0;
   // fp32 path scratch
   size_t off_f32_a = 0, off_f32_b = 0, off_f32_c = 0;
   size_t total = 0;

@@ -75,6 +75,11 @@ struct EpiCtx {
   int stage_bytes;            // bytes of the ring
   uint64_t* aux_bar;          // spare mbarrier (count 1), phase 0 unused so far
   const CUtensorMap* tA1;     // A-operand source-1 tensor map
+  // K-split bookkeeping (non-persistent kernel): the output tile's index, the
+  // number of splits, and a shared-memory word for the last-split decision.
+  int tile_id;
+  int splits;
+  uint32_t* flag;
 };
 
 // 16-column TMEM load (for tiles whose width is an odd multiple of 16).
@@ -270,6 +275,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     c.stage_bytes = STAGES * Cfg::STAGE_BYTES;
     c.aux_bar = aux;
     c.tA1 = &tA1;
+    c.tile_id = m_tile * (int)gridDim.x + n_tile;
+    c.splits = (int)gridDim.z;
+    c.flag = tmem_slot + 1;
     Epi::template run<Cfg::BN>(ep, st, c, geom);
   }
 
@@ -459,6 +467,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       c.stage_bytes = 0;
       c.aux_bar = nullptr;
       c.tA1 = &tA1;
+      c.tile_id = t;
+      c.splits = 1;
+      c.flag = nullptr;
       Epi::template run<Cfg::BN>(ep, st, c, geom);
       tc_fence_before();
       __syncwarp();
@@ -665,6 +676,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       c.stage_bytes = 0;
       c.aux_bar = nullptr;
       c.tA1 = &tA1;
+      c.tile_id = t;
+      c.splits = 1;
+      c.flag = nullptr;
       Epi::template run<Cfg::BN>(ep, st, c, geom);
       tc_fence_before();
       __syncwarp();
@@ -749,5 +763,26 @@ struct EpiPartialF32 {
     });
   }
 };
+
+// ------------------------------------------------------------------ K-split finish
+//
+// With the K loop split over blockIdx.z, an epilogue whose per-tile result is
+// small can finish it in place: every split CTA stores its partial, then
+// counts itself in the tile's counter (zeroed before the launch); the CTA that
+// completes the count re-reads all partials in split order (so the result does
+// not depend on which CTA came last). Called by all 128 epilogue threads after
+// their partial stores; true in the CTA that completes the tile.
+__device__ __forceinline__ bool split_arrive_last(const EpiCtx& c, unsigned int* counters) {
+  __threadfence();
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  if (c.row == 0) {
+    const unsigned int old = atomicAdd(&counters[c.tile_id], 1u);
+    *c.flag = (old == (unsigned int)(c.splits - 1)) ? 1u : 0u;
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  const bool last = *reinterpret_cast<volatile uint32_t*>(c.flag) != 0u;
+  if (last) __threadfence();
+  return last;
+}
 
 }  // namespace dora
