@@ -17,6 +17,7 @@
 #include <atomic>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "dora_internal.h"
 #include "gemm_sm100.cuh"
@@ -79,6 +80,24 @@ static bool make_map(CUtensorMap* map, const Mat& m, int box_outer, const char* 
   return true;
 }
 
+// Launch with programmatic stream serialization so the kernel's prologue can
+// overlap the previous kernel's tail (see pdl_wait / pdl_trigger).
+template <class... KArgs, class... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 static dora_status_t gemm_status(cudaError_t e, const char* where) {
   if (e == cudaSuccess) return DORA_OK;
   set_error(std::string(where) + ": " + cudaGetErrorString(e) + (t_detail.empty() ? "" : " [" + t_detail + "]"));
@@ -138,9 +157,9 @@ static cudaError_t launch_gemm(const GemmArgs& g, const typename Epi::Params& ep
   }
   {
     ProfRange pr(g.name, st);
-    kern<<<grid, kGemmThreads, Cfg::SMEM_BYTES, st>>>(ta0, ta1, tb0, tb1, geom, ep);
+    e = launch_pdl(kern, grid, dim3(kGemmThreads), Cfg::SMEM_BYTES, st, ta0, ta1, tb0, tb1, geom, ep);
   }
-  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess)
     t_detail = "launch grid (" + std::to_string(grid.x) + "," + std::to_string(grid.y) + "," +
                std::to_string(grid.z) + ") smem " + std::to_string(Cfg::SMEM_BYTES);
@@ -178,9 +197,9 @@ static cudaError_t launch_gemm_persistent(const GemmArgs& g, const typename Epi:
   }
   {
     ProfRange pr(g.name, st);
-    kern<<<grid, kGemmThreads, Cfg::SMEM_BYTES, st>>>(ta0, ta1, tb0, tb1, geom, ep);
+    e = launch_pdl(kern, dim3(grid), dim3(kGemmThreads), Cfg::SMEM_BYTES, st, ta0, ta1, tb0, tb1, geom, ep);
   }
-  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) t_detail = "persistent launch grid " + std::to_string(grid);
   return e;
 }
@@ -215,9 +234,10 @@ static cudaError_t launch_gemm_pair(const GemmArgs& g, const typename Epi::Param
   }
   {
     ProfRange pr(g.name, st);
-    kern<<<(unsigned)(2 * pairs), kGemmThreads, Cfg::SMEM_BYTES, st>>>(ta0, ta1, tb0, tb1, geom, ep);
+    e = launch_pdl(kern, dim3((unsigned)(2 * pairs)), dim3(kGemmThreads), Cfg::SMEM_BYTES, st, ta0, ta1, tb0,
+                   tb1, geom, ep);
   }
-  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) t_detail = "pair launch, " + std::to_string(pairs) + " clusters of 2";
   return e;
 }
@@ -402,6 +422,8 @@ static cudaError_t norm_gemm(int bn, const GemmArgs& g, const EpiNorm::Params& e
 __global__ void reduce_splits_bf16_kernel(const float* __restrict__ part, int splits, long long split_stride,
                                           int M, int N, float alpha, __nv_bfloat16* __restrict__ out,
                                           long long ldo, int transpose) {
+  pdl_trigger();
+  pdl_wait();
   const int ng = N / 4;
   const long long total = (long long)M * ng;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
@@ -438,6 +460,8 @@ __global__ void reduce_splits_bf16_kernel(const float* __restrict__ part, int sp
 // hi = bf16(x) and lo = bf16(x - hi), so hi + lo carries x to about 2^-17.
 __global__ void gram_finalize_kernel(const float* __restrict__ part, int splits, int r, int rp, float half_s,
                                      __nv_bfloat16* __restrict__ gs2) {
+  pdl_trigger();
+  pdl_wait();
   const long long total = (long long)r * 2 * rp;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
@@ -476,6 +500,8 @@ __global__ void __launch_bounds__(256) compose_bwd_bf16_kernel(const __nv_bfloat
                                                                float* __restrict__ part,
                                                                unsigned int* __restrict__ counters,
                                                                float* __restrict__ dm, int T, int d_out) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[8][64];
   __shared__ unsigned int last_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -543,9 +569,10 @@ static cudaError_t reduce_splits(const float* part, const Split& sp, long long s
   const int threads = 256;
   const long long blocks = std::min<long long>(ceil_div(total, threads), 148LL * 16);
   ProfRange pr(name, st);
-  reduce_splits_bf16_kernel<<<(unsigned)std::max<long long>(blocks, 1), threads, 0, st>>>(
-      part, sp.splits, split_stride, M, N, alpha, out, ldo, transpose ? 1 : 0);
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(reduce_splits_bf16_kernel, dim3((unsigned)std::max<long long>(blocks, 1)),
+                             dim3(threads), 0, st, part, sp.splits, split_stride, M, N, alpha, out, ldo,
+                             transpose ? 1 : 0);
+  return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
 // Narrow GEMM (N = r) with an alpha-scaled bf16 result: direct store when the
@@ -594,8 +621,9 @@ dora_status_t bf16_norm(const dora_desc_t& d, const Plan& p, const void* W0, con
     if (e != cudaSuccess) return gemm_status(e, "dora_norm: Gram");
     const long long total = (long long)r * 2 * rp;
     ProfRange pr("gram_finalize", st);
-    gram_finalize_kernel<<<(unsigned)std::min<long long>(ceil_div(total, 256), 2048), 256, 0, st>>>(
-        gram_part, p.gram.splits, r, rp, 0.5f * d.s, gs);
+    e = launch_pdl(gram_finalize_kernel, dim3((unsigned)std::min<long long>(ceil_div(total, 256), 2048)), dim3(256),
+                   0, st, (const float*)gram_part, p.gram.splits, r, rp, 0.5f * d.s, gs);
+    if (e != cudaSuccess) return cuda_status(e, "dora_norm: Gram finalize");
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_status(e, "dora_norm: Gram finalize");
   }
@@ -686,12 +714,11 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     dim3 grid(col_tiles, (unsigned)p.dm_rowblocks);
     {
       ProfRange pr("compose_bwd", st);
-      compose_bwd_bf16_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(dy),
-                                                    reinterpret_cast<const __nv_bfloat16*>(pre), g, C, dz, dm_part,
-                                                    ctr, dm, Ti, d_out);
+      cudaError_t e = launch_pdl(compose_bwd_bf16_kernel, grid, dim3(256), 0, st,
+                                 reinterpret_cast<const __nv_bfloat16*>(dy), reinterpret_cast<const __nv_bfloat16*>(pre),
+                                 g, C, dz, dm_part, ctr, dm, Ti, d_out);
+      if (e != cudaSuccess) return cuda_status(e, "dora_backward: compose backward");
     }
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_status(e, "dora_backward: compose backward");
   }
   // du = s dz B  (B read MN-major: K = d_out rows, N = r contiguous)
   {

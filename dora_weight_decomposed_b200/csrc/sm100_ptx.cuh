@@ -34,6 +34,17 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 __device__ __forceinline__ void flag_timeout() { atomicOr(&g_device_status, DORA_DEVICE_TIMEOUT); }
 
+// ---------------------------------------------------------------- dependent launches
+//
+// Kernels launched with programmatic stream serialization: pdl_trigger lets
+// the next kernel in the stream start launching once every CTA of this grid
+// has started (no CTA of this grid can then be left waiting for an SM);
+// pdl_wait blocks until the previous grid has completed and its memory
+// writes are visible. Every kernel here calls pdl_wait before its first
+// global-memory access. Both are no-ops without a programmatic dependency.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
