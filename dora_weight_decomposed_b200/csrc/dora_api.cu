@@ -54,6 +54,51 @@ static Split choose_split(int64_t tiles, int64_t kb, int sms, double kb_bytes, d
   return best;
 }
 
+// Tile width and K split of a narrow GEMM (M x N with N = r, long K) on the
+// one-CTA kernel, by a time model in microseconds: a k-block of a 128 x bn
+// tile takes the longer of its MMAs (2 clocks per tile column) and bringing
+// its (128 + bn) x 128 operand bytes into the SM (~100 bytes per clock), at
+// ~1.9 GHz; each wave of CTAs (one per SM) adds a fixed 2 us; a split K loop
+// adds the fp32 partials' write and read at ~3 TB/s and a 4 us reduction
+// launch. Wider tiles re-read the long operand less; narrower tiles and
+// splits fill more SMs.
+struct NarrowChoice {
+  int bn = 64;
+  Split split;
+};
+
+static NarrowChoice choose_narrow(int64_t M, int64_t N, int64_t K, bool b_mn, int sms) {
+  static const int kCandK[] = {16, 32, 64, 128, 192, 256, 384, 512};
+  static const int kCandMN[] = {64, 128, 192, 256, 384, 512};
+  const int* cand = b_mn ? kCandMN : kCandK;
+  const int ncand = b_mn ? 6 : 8;
+  const int64_t kb = std::max<int64_t>(cdiv(K, 64), 1);
+  NarrowChoice best;
+  double best_t = 1e300;
+  for (int ci = 0; ci < ncand; ++ci) {
+    const int bn = cand[ci];
+    if (ci > 0 && cand[ci - 1] >= N) break;  // wider than needed
+    const int64_t tiles = cdiv(M, 128) * cdiv(N, bn);
+    for (int64_t ns = 1; ns <= std::min<int64_t>(kb, 32); ++ns) {
+      const int64_t kps = cdiv(kb, ns);
+      const int64_t splits = cdiv(kb, kps);
+      if (splits != ns) continue;
+      const int64_t waves = cdiv(tiles * splits, sms);
+      const double kb_clk = std::max(2.0 * bn, (128.0 + bn) * 1.28);
+      const double t_mma = (double)kps * kb_clk / 1900.0;
+      double t = (double)waves * (t_mma + 2.0);
+      if (splits > 1) t += (double)splits * M * N * 8.0 / 3.0e6 + 4.0;
+      if (t < best_t - 1e-9) {
+        best_t = t;
+        best.bn = bn;
+        best.split.splits = (int)splits;
+        best.split.kb_per_split = (int)kps;
+      }
+    }
+  }
+  return best;
+}
+
 Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
   Plan p;
   p.sms = device_sm_count();
@@ -82,23 +127,27 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
       p.zero_bytes = (size_t)cdiv(d_out, 128) * 4;
       p.off_ctr = take(p.zero_bytes);
     } else if (op == DORA_OP_FORWARD && T > 0) {
-      p.u_bn = bn_narrow_k(r);
-      p.u = choose_split(cdiv(T, 128), cdiv(d_in, 64), p.sms, kbB * (128 + p.u_bn), 128.0 * p.u_bn,
-                         (double)T * r);
+      const NarrowChoice u = choose_narrow(T, r, d_in, false, p.sms);
+      p.u_bn = u.bn;
+      p.u = u.split;
       if (p.u.splits > 1) p.off_u_part = take((size_t)p.u.splits * T * r * 4);
       p.off_su = take((size_t)T * r * 2);
     } else if (op == DORA_OP_BACKWARD && T > 0) {
       p.off_dz = take((size_t)T * d_out * 2);
       p.dm_rowblocks = (int)cdiv(T, 256);
       p.off_dm_part = take((size_t)p.dm_rowblocks * d_out * 4);
-      p.r_bn_mn = bn_narrow_mn(r);
-      const double kb_mn = kbB * (128 + p.r_bn_mn);
-      p.du = choose_split(cdiv(T, 128), cdiv(d_out, 64), p.sms, kb_mn, 128.0 * p.r_bn_mn, (double)T * r);
+      const NarrowChoice du = choose_narrow(T, r, d_out, true, p.sms);
+      p.du_bn = du.bn;
+      p.du = du.split;
       if (p.du.splits > 1) p.off_du_part = take((size_t)p.du.splits * T * r * 4);
       p.off_du = take((size_t)T * r * 2);
-      p.dB = choose_split(cdiv(d_out, 128), cdiv(T, 64), p.sms, kb_mn, 128.0 * p.r_bn_mn, (double)d_out * r);
+      const NarrowChoice dB = choose_narrow(d_out, r, T, true, p.sms);
+      p.dB_bn = dB.bn;
+      p.dB = dB.split;
       if (p.dB.splits > 1) p.off_dB_part = take((size_t)p.dB.splits * d_out * r * 4);
-      p.dA = choose_split(cdiv(d_in, 128), cdiv(T, 64), p.sms, kb_mn, 128.0 * p.r_bn_mn, (double)d_in * r);
+      const NarrowChoice dA = choose_narrow(d_in, r, T, true, p.sms);
+      p.dA_bn = dA.bn;
+      p.dA = dA.split;
       if (p.dA.splits > 1) p.off_dA_part = take((size_t)p.dA.splits * d_in * r * 4);
       // counters of the dm column strips, zeroed by one memset per call
       p.zero_bytes = (size_t)cdiv(d_out, 64) * 4;

@@ -222,9 +222,11 @@ static cudaError_t launch_gemm_pair(const GemmArgs& g, const typename Epi::Param
     ta1 = ta0;
     tb1 = tb0;
   }
-  GemmGeom geom{g.M, g.N, kb0, kb1, kb0 + kb1, g.a1_kwrap};
-  const long long tiles = ceil_div(g.N, Cfg::BN) * ceil_div(g.M, 2 * kBM);
-  const long long pairs = std::max<long long>(1, std::min<long long>(tiles, sms / 2));
+  const int kps = g.split.kb_per_split > 0 ? g.split.kb_per_split : kb0 + kb1;
+  GemmGeom geom{g.M, g.N, kb0, kb1, kps, g.a1_kwrap};
+  const long long splits = ceil_div(std::max(kb0 + kb1, 1), kps);
+  const long long items = ceil_div(g.N, Cfg::BN) * ceil_div(g.M, 2 * kBM) * splits;
+  const long long pairs = std::max<long long>(1, std::min<long long>(items, sms / 2));
   auto kern = gemm_sm100_pair_kernel<Cfg, Epi>;
   static std::atomic<unsigned long long> smem_set{0};
   cudaError_t e = set_smem_once(smem_set, kern, Cfg::SMEM_BYTES);
@@ -250,6 +252,7 @@ static cudaError_t gemm_bn(int bn, const GemmArgs& g, const typename Epi::Params
   }
   if (bn == 64) return launch_gemm<GemmCfg<64, A_MN, B_MN>, Epi>(g, ep, st);
   if (bn == 128) return launch_gemm<GemmCfg<128, A_MN, B_MN>, Epi>(g, ep, st);
+  if (bn == 192) return launch_gemm<GemmCfg<192, A_MN, B_MN>, Epi>(g, ep, st);
   if (bn == 256) return launch_gemm<GemmCfg<256, A_MN, B_MN>, Epi>(g, ep, st);
   if (bn == 384) return launch_gemm<GemmCfg<384, A_MN, B_MN>, Epi>(g, ep, st);
   if (bn == 512) return launch_gemm<GemmCfg<512, A_MN, B_MN>, Epi>(g, ep, st);
@@ -382,7 +385,7 @@ struct EpiCompose {
       __nv_bfloat16* yrow = p.y + (long long)c.m * p.ldo + n;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        if (n + 8 * j < g.N) {
+        if (col + 8 * j < BN && n + 8 * j < g.N) {
           const float4 ga = __ldg(reinterpret_cast<const float4*>(p.gm1 + n + 8 * j));
           const float4 gb = __ldg(reinterpret_cast<const float4*>(p.gm1 + n + 8 * j + 4));
           const float gm[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
@@ -577,9 +580,12 @@ static cudaError_t reduce_splits(const float* part, const Split& sp, long long s
 
 // Narrow GEMM (N = r) with an alpha-scaled bf16 result: direct store when the
 // K loop is not split, else fp32 partials summed by reduce_splits.
+// Narrow GEMM (N = r) with an alpha-scaled bf16 result: direct store when the
+// K loop is not split, else fp32 partials summed by reduce_splits.
 template <bool A_MN, bool B_MN>
 static cudaError_t narrow_gemm(int bn, const GemmArgs& g, float alpha, __nv_bfloat16* out, long long ldo,
-                               bool transpose, float* part, const char* reduce_name, cudaStream_t st) {
+                               bool transpose, float* part, const char* reduce_name, int sms, cudaStream_t st) {
+  (void)sms;
   if (g.split.splits == 1) {
     EpiStoreBF16::Params p{out, ldo, alpha, transpose ? 1 : 0};
     return gemm_bn<A_MN, B_MN, EpiStoreBF16>(bn, g, p, st);
@@ -666,7 +672,7 @@ dora_status_t bf16_forward(const dora_desc_t& d, const Plan& p, int64_t T, const
   ua.split = p.u;
   ua.name = "u_gemm";
   cudaError_t e = narrow_gemm<false, false>(p.u_bn, ua, d.s, su, r, false, reinterpret_cast<float*>(ws + p.off_u_part),
-                                "u_reduce", st);
+                                "u_reduce", p.sms, st);
   if (e != cudaSuccess) return gemm_status(e, "dora_forward: LoRA down projection");
 
   // pre = [x | su] [W0 | B]^T, y = pre + gm1 * pre
@@ -730,8 +736,8 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.N = r;
     a.split = p.du;
     a.name = "du_gemm";
-    cudaError_t e = narrow_gemm<false, true>(p.r_bn_mn, a, d.s, du, r, false,
-                                             reinterpret_cast<float*>(ws + p.off_du_part), "du_reduce", st);
+    cudaError_t e = narrow_gemm<false, true>(p.du_bn, a, d.s, du, r, false,
+                                             reinterpret_cast<float*>(ws + p.off_du_part), "du_reduce", p.sms, st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: du");
   }
   // dB = dz^T su  (both token-major: K = T)
@@ -744,8 +750,8 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.N = r;
     a.split = p.dB;
     a.name = "dB_gemm";
-    cudaError_t e = narrow_gemm<true, true>(p.r_bn_mn, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dB), r, false,
-                                            reinterpret_cast<float*>(ws + p.off_dB_part), "dB_reduce", st);
+    cudaError_t e = narrow_gemm<true, true>(p.dB_bn, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dB), r, false,
+                                            reinterpret_cast<float*>(ws + p.off_dB_part), "dB_reduce", p.sms, st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: dB");
   }
   // dA^T = x^T du, stored transposed into dA [r x d_in]
@@ -758,8 +764,8 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.N = r;
     a.split = p.dA;
     a.name = "dA_gemm";
-    cudaError_t e = narrow_gemm<true, true>(p.r_bn_mn, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dA), d_in, true,
-                                            reinterpret_cast<float*>(ws + p.off_dA_part), "dA_reduce", st);
+    cudaError_t e = narrow_gemm<true, true>(p.dA_bn, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dA), d_in, true,
+                                            reinterpret_cast<float*>(ws + p.off_dA_part), "dA_reduce", p.sms, st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: dA");
   }
   // dx = [dz | du] [W0 ; A]  (W0 and A read MN-major: K rows, N = d_in contiguous)

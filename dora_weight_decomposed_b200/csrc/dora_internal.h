@@ -31,7 +31,7 @@ struct Plan {
   // backward
   int dm_rowblocks = 0;
   Split du, dB, dA;
-  int r_bn_mn = 0;
+  int du_bn = 0, dB_bn = 0, dA_bn = 0;
   size_t off_dz = 0, off_dm_part = 0, off_du_part = 0, off_du = 0, off_dB_part = 0, off_dA_part = 0;
   // split counters (+ padding that must start at zero), cleared by one memset per call
   size_t off_ctr = 0, zero_bytes = 0;

@@ -45,7 +45,7 @@ struct GemmCfg {
   static constexpr bool B_MN = B_MN_;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 512, "BN");
   static_assert(!B_MN || BN % 64 == 0, "MN-major B tiles are whole 64-wide swizzle chunks");
-  static_assert(BN <= 128 || BN % 128 == 0, "BN above 128 must be a multiple of 128");
+  static_assert(BN <= 128 || BN % 64 == 0, "BN above 128 must be a multiple of 64");
   static constexpr int A_BYTES = kBM * kBK * 2;
   static constexpr int B_BYTES = BN * kBK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -58,7 +58,7 @@ struct GemmCfg {
   static constexpr int MMA_N0 = BN <= 256 ? BN : 256;
   static constexpr int MMA_N1 = BN <= 256 ? 0 : BN - 256;
   // TMA boxes: K-major B uses boxes of B_BOX rows; MN-major uses 64x64 chunks.
-  static constexpr int B_BOX = B_MN ? 64 : (BN <= 128 ? BN : 128);
+  static constexpr int B_BOX = B_MN ? 64 : (BN <= 128 ? BN : (BN % 128 == 0 ? 128 : 64));
   static constexpr int B_LOADS = BN / B_BOX;
 };
 
@@ -503,9 +503,15 @@ struct PairCfg {
   static constexpr int BN = BN_;
   static constexpr bool A_MN = A_MN_;
   static constexpr bool B_MN = B_MN_;
-  static constexpr int BH = BN / 2;  // B rows (N) staged by each CTA
-  static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "pair tile N");
-  static_assert(!B_MN || BH % 64 == 0, "MN-major B halves are whole 64-wide chunks");
+  static_assert(BN % 32 == 0 && BN >= 64 && BN <= 512, "pair tile N");
+  // N above 256 takes two MMAs: columns [0, N0) and [N0, BN). Each CTA stages
+  // half of each MMA's B columns: H0 rows for the first, then H1 for the second.
+  static constexpr int N0 = BN <= 256 ? BN : 256;
+  static constexpr int N1 = BN - N0;
+  static constexpr int H0 = N0 / 2;
+  static constexpr int H1 = N1 / 2;
+  static constexpr int BH = H0 + H1;
+  static_assert(!B_MN || (H0 % 64 == 0 && H1 % 64 == 0), "MN-major B halves are whole 64-wide chunks");
   static constexpr int A_BYTES = kBM * kBK * 2;
   static constexpr int B_BYTES = BH * kBK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -513,11 +519,18 @@ struct PairCfg {
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
-  static constexpr int B_BOX = B_MN ? 64 : (BH <= 128 ? BH : 128);
-  static constexpr int B_LOADS = BH / B_BOX;
-  static constexpr uint32_t ACC_COLS = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
+  static constexpr int B_BOX = B_MN ? 64 : (H1 == 0 ? H0 : (H0 == H1 ? H0 : 64));
+  static constexpr int B0_LOADS = H0 / B_BOX;
+  static constexpr int B1_LOADS = H1 / B_BOX;
+  // Offset of the second MMA's B half inside the stage.
+  static constexpr uint32_t B1_OFFSET = B_MN ? (uint32_t)(H0 / 64) * 8192u : (uint32_t)H0 * 128u;
+  // Two accumulators (epilogue overlaps the next item's MMAs) when N <= 256.
+  static constexpr int NUM_ACC = BN <= 256 ? 2 : 1;
+  static constexpr uint32_t ACC_COLS = BN <= 64 ? 64 : BN <= 128 ? 128 : BN <= 256 ? 256 : 512;
+  static constexpr uint32_t TMEM_COLS = NUM_ACC * ACC_COLS > 512 ? 512 : NUM_ACC * ACC_COLS;
 };
 
+// Work items are (output tile, K split) pairs: item = tile * splits + split.
 template <class Cfg, class Epi>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_sm100_pair_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tA1,
@@ -525,8 +538,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                            const GemmGeom geom, const typename Epi::Params ep) {
   static_assert(!Epi::kReadsA, "pair epilogues do not read A stages");
   constexpr int STAGES = Cfg::STAGES;
+  constexpr int NACC = Cfg::NUM_ACC;
   constexpr uint32_t ACC_COLS = Cfg::ACC_COLS;
-  constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
+  constexpr uint32_t TMEM_COLS = Cfg::TMEM_COLS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
@@ -542,8 +556,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const int npairs = gridDim.x >> 1;
   const int m_tiles = (geom.M + 2 * kBM - 1) / (2 * kBM);
   const int n_tiles = (geom.N + Cfg::BN - 1) / Cfg::BN;
-  const int tiles = m_tiles * n_tiles;
-  const int nkb = geom.kb0 + geom.kb1;
+  const int kb_total = geom.kb0 + geom.kb1;
+  const int kps = geom.kb_per_split;
+  const int splits = (kb_total + kps - 1) / kps;
+  const int items = m_tiles * n_tiles * splits;
 
   if (threadIdx.x == 0) {
 #pragma unroll 1
@@ -582,13 +598,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int it = 0;
       bool ok = true;
 #pragma unroll 1
-      for (int t = pair; t < tiles && ok; t += npairs) {
+      for (int item = pair; item < items && ok; item += npairs) {
+        const int t = item / splits, split = item - t * splits;
         int tm, tn;
         tile_coords(t, m_tiles, n_tiles, tm, tn);
         const int m0 = tm * 2 * kBM + (int)rank * kBM;
-        const int nb = tn * Cfg::BN + (int)rank * Cfg::BH;
+        const int nb0 = tn * Cfg::BN + (int)rank * Cfg::H0;
+        const int nb1 = tn * Cfg::BN + Cfg::N0 + (int)rank * Cfg::H1;
+        const int kb_end = min(kb_total, (split + 1) * kps);
 #pragma unroll 1
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
+        for (int kb = split * kps; kb < kb_end; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
           if (!mbar_wait(&empty[s], ph ^ 1u)) {
@@ -611,18 +630,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             tma_load_2d_pair(sa + 8192, ta, fb, m0 + 64, k0a);
           }
 #pragma unroll
-          for (int j = 0; j < Cfg::B_LOADS; ++j) {
+          for (int j = 0; j < Cfg::B0_LOADS; ++j) {
             if (!Cfg::B_MN)
-              tma_load_2d_pair(sb + j * Cfg::B_BOX * 128, tb, fb, k0, nb + j * Cfg::B_BOX);
+              tma_load_2d_pair(sb + j * Cfg::B_BOX * 128, tb, fb, k0, nb0 + j * Cfg::B_BOX);
             else
-              tma_load_2d_pair(sb + j * 8192, tb, fb, nb + j * 64, k0);
+              tma_load_2d_pair(sb + j * 8192, tb, fb, nb0 + j * 64, k0);
+          }
+#pragma unroll
+          for (int j = 0; j < Cfg::B1_LOADS; ++j) {
+            if (!Cfg::B_MN)
+              tma_load_2d_pair(sb + Cfg::B1_OFFSET + j * Cfg::B_BOX * 128, tb, fb, k0, nb1 + j * Cfg::B_BOX);
+            else
+              tma_load_2d_pair(sb + Cfg::B1_OFFSET + j * 8192, tb, fb, nb1 + j * 64, k0);
           }
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(2 * kBM, Cfg::BN, Cfg::A_MN, Cfg::B_MN);
+      constexpr uint32_t idesc0 = idesc_bf16_f32(2 * kBM, Cfg::N0, Cfg::A_MN, Cfg::B_MN);
+      constexpr uint32_t idesc1 = idesc_bf16_f32(2 * kBM, Cfg::N1 > 0 ? Cfg::N1 : 16, Cfg::A_MN, Cfg::B_MN);
       constexpr uint32_t a_kstep = Cfg::A_MN ? 2048u : 32u;
       constexpr uint32_t b_kstep = Cfg::B_MN ? 2048u : 32u;
       constexpr uint32_t a_lbo = Cfg::A_MN ? 8192u : 16u;
@@ -630,14 +657,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int it = 0, j = 0;
       bool ok = true;
 #pragma unroll 1
-      for (int t = pair; t < tiles && ok; t += npairs, ++j) {
-        const int b = j & 1;
-        const uint32_t uph = (uint32_t)(j >> 1) & 1u;
+      for (int item = pair; item < items && ok; item += npairs, ++j) {
+        const int t = item / splits, split = item - t * splits;
+        const int b = j % NACC;
+        const uint32_t uph = (uint32_t)(j / NACC) & 1u;
         if (!mbar_wait(&acce[b], uph ^ 1u)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)b * ACC_COLS;
+        const int kb_begin = split * kps;
+        const int kb_end = min(kb_total, kb_begin + kps);
+        (void)t;
 #pragma unroll 1
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
+        for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
           if (!mbar_wait(&full[s], ph)) {
@@ -650,8 +681,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t ad = sdesc_sw128(sa + kk * a_kstep, a_lbo, 1024u);
-            const uint64_t bd = sdesc_sw128(sb + kk * b_kstep, b_lbo, 1024u);
-            umma_bf16_pair(d_tmem, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            const uint64_t bd0 = sdesc_sw128(sb + kk * b_kstep, b_lbo, 1024u);
+            const uint32_t acc = (kb > kb_begin || kk > 0) ? 1u : 0u;
+            umma_bf16_pair(d_tmem, ad, bd0, idesc0, acc);
+            if (Cfg::N1 > 0) {
+              const uint64_t bd1 = sdesc_sw128(sb + Cfg::B1_OFFSET + kk * b_kstep, b_lbo, 1024u);
+              umma_bf16_pair(d_tmem + (uint32_t)Cfg::N0, ad, bd1, idesc1, acc);
+            }
           }
           umma_commit_pair(&empty[s], 0x3);
         }
@@ -664,26 +700,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     typename Epi::RowState st{};
     int j = 0;
 #pragma unroll 1
-    for (int t = pair; t < tiles; t += npairs, ++j) {
-      const int b = j & 1;
-      const uint32_t uph = (uint32_t)(j >> 1) & 1u;
+    for (int item = pair; item < items; item += npairs, ++j) {
+      const int t = item / splits, split = item - t * splits;
+      const int b = j % NACC;
+      const uint32_t uph = (uint32_t)(j / NACC) & 1u;
       if (!mbar_wait(&accf[b], uph)) break;
       tc_fence_after();
       int tm, tn;
       tile_coords(t, m_tiles, n_tiles, tm, tn);
+      const int kb_begin = split * kps;
       EpiCtx c;
       c.taddr = tmem + (uint32_t)b * ACC_COLS + ((uint32_t)(q * 32) << 16);
       c.row = row;
       c.m = tm * 2 * kBM + (int)rank * kBM + row;
       c.n0 = tn * Cfg::BN;
-      c.split = 0;
-      c.has_acc = nkb > 0;
+      c.split = split;
+      c.has_acc = min(kb_total, kb_begin + kps) > kb_begin;
       c.stage_smem = nullptr;
       c.stage_bytes = 0;
       c.aux_bar = nullptr;
       c.tA1 = &tA1;
       c.tile_id = t;
-      c.splits = 1;
+      c.splits = splits;
       c.flag = nullptr;
       Epi::template run<Cfg::BN>(ep, st, c, geom);
       tc_fence_before();
@@ -731,15 +769,17 @@ struct EpiStoreBF16 {
       if (!row_ok) return;
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] *= p.alpha;
+      // A 16-wide tile is visited as a zero-padded 32-column chunk: stores stop
+      // at the tile's own width as well as at N.
       if (!p.transpose) {
         __nv_bfloat16* dst = p.out + (long long)c.m * p.ldo + n;
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          if (n + 8 * j < g.N) store_bf16x8(dst + 8 * j, v + 8 * j);
+          if (col + 8 * j < BN && n + 8 * j < g.N) store_bf16x8(dst + 8 * j, v + 8 * j);
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-          if (n + i < g.N) p.out[(long long)(n + i) * p.ldo + c.m] = __float2bfloat16_rn(v[i]);
+          if (col + i < BN && n + i < g.N) p.out[(long long)(n + i) * p.ldo + c.m] = __float2bfloat16_rn(v[i]);
       }
     });
   }
@@ -764,7 +804,7 @@ struct EpiPartialF32 {
       if (!row_ok) return;
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        if (n + 4 * j < g.N)
+        if (col + 4 * j < BN && n + 4 * j < g.N)
           *reinterpret_cast<float4*>(base + n + 4 * j) = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
     });
   }
