@@ -54,40 +54,79 @@ static Split choose_split(int64_t tiles, int64_t kb, int sms, double kb_bytes, d
   return best;
 }
 
-// Tile width and K split of a narrow GEMM (M x N with N = r, long K) on the
-// one-CTA kernel, by a time model in microseconds: a k-block of a 128 x bn
-// tile takes the longer of its MMAs (2 clocks per tile column) and bringing
-// its (128 + bn) x 128 operand bytes into the SM (~100 bytes per clock), at
-// ~1.9 GHz; each wave of CTAs (one per SM) adds a fixed 2 us; a split K loop
-// adds the fp32 partials' write and read at ~3 TB/s and a 4 us reduction
-// launch. Wider tiles re-read the long operand less; narrower tiles and
-// splits fill more SMs.
+// Tile width and K split of a narrow GEMM (M x N with N = r, long K) on CTA
+// pairs (256-row tiles), by a time model in microseconds at ~1.9 GHz:
+//  - a k-block takes the longer of its MMAs (2 clocks per tile column) and
+//    bringing each CTA's (128 + bn/2) x 128 operand bytes in (~58 bytes per
+//    clock per SM, the TMA rate the main loops sustain);
+//  - the epilogue stores a 128 x bn tile per CTA: bf16 directly (~17 GB/s per
+//    SM) or, when K is split, fp32 partials by TMA (~100 GB/s per SM);
+//  - each wave of pairs (one per two SMs) adds a fixed 2 us;
+//  - a split K loop adds the reduction pass over all partials (~4.5 TB/s)
+//    and its launch (4 us).
 struct NarrowChoice {
-  int bn = 64;
+  int bn = 128;
   Split split;
+  bool pair = true;
 };
 
-static NarrowChoice choose_narrow(int64_t M, int64_t N, int64_t K, bool b_mn, int sms) {
+// The same on single CTAs (128-row tiles, operand bytes (128 + bn) x 128 per
+// k-block), which measured faster for dB and dA (K = T, both operands
+// token-major): 128 x 192 tiles there keep every SM busy without a K split.
+static NarrowChoice choose_narrow_1cta(int64_t M, int64_t N, int64_t K, bool b_mn, int sms) {
   static const int kCandK[] = {16, 32, 64, 128, 192, 256, 384, 512};
   static const int kCandMN[] = {64, 128, 192, 256, 384, 512};
   const int* cand = b_mn ? kCandMN : kCandK;
   const int ncand = b_mn ? 6 : 8;
   const int64_t kb = std::max<int64_t>(cdiv(K, 64), 1);
   NarrowChoice best;
+  best.pair = false;
   double best_t = 1e300;
   for (int ci = 0; ci < ncand; ++ci) {
     const int bn = cand[ci];
-    if (ci > 0 && cand[ci - 1] >= N) break;  // wider than needed
+    if (ci > 0 && cand[ci - 1] >= N) break;
     const int64_t tiles = cdiv(M, 128) * cdiv(N, bn);
+    const double kb_clk = std::max(2.0 * bn, (128.0 + bn) * 1.28);
     for (int64_t ns = 1; ns <= std::min<int64_t>(kb, 32); ++ns) {
       const int64_t kps = cdiv(kb, ns);
       const int64_t splits = cdiv(kb, kps);
       if (splits != ns) continue;
       const int64_t waves = cdiv(tiles * splits, sms);
-      const double kb_clk = std::max(2.0 * bn, (128.0 + bn) * 1.28);
-      const double t_mma = (double)kps * kb_clk / 1900.0;
-      double t = (double)waves * (t_mma + 2.0);
+      double t = (double)waves * ((double)kps * kb_clk / 1900.0 + 2.0);
       if (splits > 1) t += (double)splits * M * N * 8.0 / 3.0e6 + 4.0;
+      if (t < best_t - 1e-9) {
+        best_t = t;
+        best.bn = bn;
+        best.split.splits = (int)splits;
+        best.split.kb_per_split = (int)kps;
+      }
+    }
+  }
+  return best;
+}
+
+static NarrowChoice choose_narrow(int64_t M, int64_t N, int64_t K, bool b_mn, int sms) {
+  static const int kCandK[] = {64, 128, 256, 384, 512};
+  static const int kCandMN[] = {128, 256, 384, 512};
+  const int* cand = b_mn ? kCandMN : kCandK;
+  const int ncand = b_mn ? 4 : 5;
+  const int64_t kb = std::max<int64_t>(cdiv(K, 64), 1);
+  const int pairs = std::max(1, sms / 2);
+  NarrowChoice best;
+  double best_t = 1e300;
+  for (int ci = 0; ci < ncand; ++ci) {
+    const int bn = cand[ci];
+    if (ci > 0 && cand[ci - 1] >= N) break;  // wider than needed
+    const int64_t tiles = cdiv(M, 256) * cdiv(N, bn);
+    const double kb_clk = std::max(2.0 * bn, (128.0 + bn / 2.0) * 128.0 / 58.0);
+    for (int64_t ns = 1; ns <= std::min<int64_t>(kb, 32); ++ns) {
+      const int64_t kps = cdiv(kb, ns);
+      const int64_t splits = cdiv(kb, kps);
+      if (splits != ns) continue;
+      const int64_t waves = cdiv(tiles * splits, pairs);
+      const double epi = splits > 1 ? 128.0 * bn * 4.0 / 1.0e5 : 128.0 * bn * 2.0 / 1.7e4;
+      double t = (double)waves * ((double)kps * kb_clk / 1900.0 + epi + 2.0);
+      if (splits > 1) t += (double)splits * M * N * 8.0 / 4.5e6 + 4.0;
       if (t < best_t - 1e-9) {
         best_t = t;
         best.bn = bn;
@@ -113,10 +152,12 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
     const double kbB = 64.0 * 2.0;  // bytes per K element pair of rows (x 64 K per k-block)
     if (op == DORA_OP_NORM) {
       const int bk = bn_narrow_k(r);
-      // The Gram GEMM is small; its fp32 partials are capped at 8 MiB.
+      // The Gram GEMM (CTA pairs, one tile column) is small: split K over the
+      // pairs, with its fp32 partials capped at 8 MiB.
+      p.gram_bn = bn_pair_k(r);
       const int64_t gram_max = std::max<int64_t>(1, (int64_t(8) << 20) / (r * r * 4));
-      p.gram = choose_split(cdiv(r, 128), cdiv(d_in, 64), p.sms, kbB * (128 + bk), 128.0 * bk, (double)r * r,
-                            gram_max);
+      p.gram = choose_split(cdiv(r, 256), cdiv(d_in, 64), p.sms / 2, kbB * (128 + p.gram_bn / 2.0), 0.0,
+                            (double)r * r, gram_max);
       p.off_gram_part = take((size_t)p.gram.splits * r * r * 4);
       p.norm = choose_split(cdiv(d_out, 128), cdiv(d_in, 64) + 2 * cdiv(r, 64), p.sms, kbB * (128 + bk), 0.0,
                             (double)d_out);
@@ -141,11 +182,11 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
       p.du = du.split;
       if (p.du.splits > 1) p.off_du_part = take((size_t)p.du.splits * T * r * 4);
       p.off_du = take((size_t)T * r * 2);
-      const NarrowChoice dB = choose_narrow(d_out, r, T, true, p.sms);
+      const NarrowChoice dB = choose_narrow_1cta(d_out, r, T, true, p.sms);
       p.dB_bn = dB.bn;
       p.dB = dB.split;
       if (p.dB.splits > 1) p.off_dB_part = take((size_t)p.dB.splits * d_out * r * 4);
-      const NarrowChoice dA = choose_narrow(d_in, r, T, true, p.sms);
+      const NarrowChoice dA = choose_narrow_1cta(d_in, r, T, true, p.sms);
       p.dA_bn = dA.bn;
       p.dA = dA.split;
       if (p.dA.splits > 1) p.off_dA_part = take((size_t)p.dA.splits * d_in * r * 4);

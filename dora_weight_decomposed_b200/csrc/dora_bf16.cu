@@ -104,6 +104,27 @@ static dora_status_t gemm_status(cudaError_t e, const char* where) {
   return DORA_ECUDA;
 }
 
+// fp32 [d2][d1][d0] array (d0 contiguous) for tiled 3-D stores of box {b0, b1, 1}, 128-byte swizzle.
+static bool make_map_f32_3d(CUtensorMap* map, void* base, int64_t d0, int64_t d1, int64_t d2, int b0, int b1) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || d0 <= 0 || d1 <= 0 || d2 <= 0) {
+    t_detail = "fp32 store map: bad extent or no encoder";
+    return false;
+  }
+  cuuint64_t dims[3] = {(cuuint64_t)d0, (cuuint64_t)d1, (cuuint64_t)d2};
+  cuuint64_t strides[2] = {(cuuint64_t)d0 * 4, (cuuint64_t)(d0 * d1) * 4};
+  cuuint32_t box[3] = {(cuuint32_t)b0, (cuuint32_t)b1, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    t_detail = "fp32 store map encode failed (CUresult " + std::to_string((int)r) + ")";
+    return false;
+  }
+  return true;
+}
+
 // ============================================================== GEMM launch
 
 struct GemmArgs {
@@ -228,16 +249,17 @@ static cudaError_t launch_gemm_pair(const GemmArgs& g, const typename Epi::Param
   const long long items = ceil_div(g.N, Cfg::BN) * ceil_div(g.M, 2 * kBM) * splits;
   const long long pairs = std::max<long long>(1, std::min<long long>(items, sms / 2));
   auto kern = gemm_sm100_pair_kernel<Cfg, Epi>;
+  constexpr int smem_bytes = PairLayout<Cfg, Epi>::SMEM_BYTES;
   static std::atomic<unsigned long long> smem_set{0};
-  cudaError_t e = set_smem_once(smem_set, kern, Cfg::SMEM_BYTES);
+  cudaError_t e = set_smem_once(smem_set, kern, smem_bytes);
   if (e != cudaSuccess) {
-    t_detail = "shared-memory attribute (" + std::to_string(Cfg::SMEM_BYTES) + " bytes)";
+    t_detail = "shared-memory attribute (" + std::to_string(smem_bytes) + " bytes)";
     return e;
   }
   {
     ProfRange pr(g.name, st);
-    e = launch_pdl(kern, dim3((unsigned)(2 * pairs)), dim3(kGemmThreads), Cfg::SMEM_BYTES, st, ta0, ta1, tb0,
-                   tb1, geom, ep);
+    e = launch_pdl(kern, dim3((unsigned)(2 * pairs)), dim3(kGemmThreads), smem_bytes, st, ta0, ta1, tb0, tb1,
+                   geom, ep);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) t_detail = "pair launch, " + std::to_string(pairs) + " clusters of 2";
@@ -375,6 +397,7 @@ struct EpiCompose {
   };
   using RowState = NoRowState;
   static constexpr bool kReadsA = false;
+  static constexpr int kStageOutBytes = 0;
   __device__ static void on_a_stage(const Params&, RowState&, const uint8_t*, bool) {}
   template <int BN>
   __device__ static void run(const Params& p, RowState&, const EpiCtx& c, const GemmGeom& g) {
@@ -458,29 +481,42 @@ __global__ void reduce_splits_bf16_kernel(const float* __restrict__ part, int sp
   }
 }
 
-// Gram finalize: x = (s/2) sum_z part[z] in fp32, written as two bf16 halves
-// Gs2[n] = [hi(x_n,0..r-1), 0 .. | lo(x_n,0..r-1), 0 ..] with rp columns each,
-// hi = bf16(x) and lo = bf16(x - hi), so hi + lo carries x to about 2^-17.
+// Gram finalize: x = (s/2) sum_z part[z] in fp32 (split order fixed), written
+// as two bf16 halves Gs2[n] = [hi(x_n,0..r-1), 0 .. | lo(x_n,0..r-1), 0 ..]
+// with rp columns each, hi = bf16(x) and lo = bf16(x - hi), so hi + lo carries
+// x to about 2^-17. Each thread takes 4 consecutive columns of one half-row.
 __global__ void gram_finalize_kernel(const float* __restrict__ part, int splits, int r, int rp, float half_s,
                                      __nv_bfloat16* __restrict__ gs2) {
   pdl_trigger();
   pdl_wait();
-  const long long total = (long long)r * 2 * rp;
+  const int qn = rp / 4;  // 4-column groups per half-row
+  const long long total = (long long)r * 2 * qn;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
-    const int n = (int)(i / (2 * rp));
-    const int k = (int)(i % (2 * rp));
-    const bool lo = k >= rp;
-    const int c = lo ? k - rp : k;
-    float v = 0.f;
+    const int n = (int)(i / (2 * qn));
+    const int qq = (int)(i % (2 * qn));
+    const bool lo = qq >= qn;
+    const int c = (lo ? qq - qn : qq) * 4;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
     if (c < r) {
-      float x = 0.f;
-      for (int z = 0; z < splits; ++z) x += part[(long long)z * r * r + (long long)n * r + c];
-      x *= half_s;
-      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-      v = lo ? x - __bfloat162float(hi) : x;
+      const float* src = part + (long long)n * r + c;
+#pragma unroll 4
+      for (int z = 0; z < splits; ++z) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(src + (long long)z * r * r));
+        x.x += v.x;
+        x.y += v.y;
+        x.z += v.z;
+        x.w += v.w;
+      }
     }
-    gs2[i] = __float2bfloat16_rn(v);
+    const float xs[4] = {half_s * x.x, half_s * x.y, half_s * x.z, half_s * x.w};
+    __nv_bfloat16 o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(xs[j]);
+      o[j] = (c + j < r) ? (lo ? __float2bfloat16_rn(xs[j] - __bfloat162float(hi)) : hi) : __float2bfloat16_rn(0.f);
+    }
+    *reinterpret_cast<uint2*>(gs2 + (long long)n * 2 * rp + (lo ? rp : 0) + c) = *reinterpret_cast<const uint2*>(o);
   }
 }
 
@@ -578,14 +614,27 @@ static cudaError_t reduce_splits(const float* part, const Split& sp, long long s
   return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
+// CTA-pair dispatch on the tile width.
+template <bool A_MN, bool B_MN, class Epi>
+static cudaError_t pair_gemm_bn(int bn, const GemmArgs& g, const typename Epi::Params& ep, int sms, cudaStream_t st) {
+  if constexpr (!B_MN) {
+    if (bn == 64) return launch_gemm_pair<PairCfg<64, A_MN, B_MN>, Epi>(g, ep, sms, st);
+  }
+  if (bn == 128) return launch_gemm_pair<PairCfg<128, A_MN, B_MN>, Epi>(g, ep, sms, st);
+  if (bn == 256) return launch_gemm_pair<PairCfg<256, A_MN, B_MN>, Epi>(g, ep, sms, st);
+  if (bn == 384) return launch_gemm_pair<PairCfg<384, A_MN, B_MN>, Epi>(g, ep, sms, st);
+  if (bn == 512) return launch_gemm_pair<PairCfg<512, A_MN, B_MN>, Epi>(g, ep, sms, st);
+  t_detail = "no pair tile of width " + std::to_string(bn);
+  return cudaErrorInvalidValue;
+}
+
 // Narrow GEMM (N = r) with an alpha-scaled bf16 result: direct store when the
-// K loop is not split, else fp32 partials summed by reduce_splits.
-// Narrow GEMM (N = r) with an alpha-scaled bf16 result: direct store when the
-// K loop is not split, else fp32 partials summed by reduce_splits.
+// K loop is not split, else fp32 partials summed in split order by
+// reduce_splits. On single CTAs the threads store the partials; on CTA pairs
+// the epilogue warps stage them for TMA stores.
 template <bool A_MN, bool B_MN>
-static cudaError_t narrow_gemm(int bn, const GemmArgs& g, float alpha, __nv_bfloat16* out, long long ldo,
-                               bool transpose, float* part, const char* reduce_name, int sms, cudaStream_t st) {
-  (void)sms;
+static cudaError_t narrow_gemm_1cta(int bn, const GemmArgs& g, float alpha, __nv_bfloat16* out, long long ldo,
+                                    bool transpose, float* part, const char* reduce_name, cudaStream_t st) {
   if (g.split.splits == 1) {
     EpiStoreBF16::Params p{out, ldo, alpha, transpose ? 1 : 0};
     return gemm_bn<A_MN, B_MN, EpiStoreBF16>(bn, g, p, st);
@@ -594,6 +643,21 @@ static cudaError_t narrow_gemm(int bn, const GemmArgs& g, float alpha, __nv_bflo
   EpiPartialF32::Params p{part, g.N, sstride};
   cudaError_t e = gemm_bn<A_MN, B_MN, EpiPartialF32>(bn, g, p, st);
   if (e != cudaSuccess) return e;
+  return reduce_splits(part, g.split, sstride, g.M, g.N, alpha, out, ldo, transpose, reduce_name, st);
+}
+
+template <bool A_MN, bool B_MN>
+static cudaError_t narrow_gemm_pair(int bn, const GemmArgs& g, float alpha, __nv_bfloat16* out, long long ldo,
+                                    bool transpose, float* part, const char* reduce_name, int sms, cudaStream_t st) {
+  if (g.split.splits == 1) {
+    EpiStoreBF16::Params p{out, ldo, alpha, transpose ? 1 : 0};
+    return pair_gemm_bn<A_MN, B_MN, EpiStoreBF16>(bn, g, p, sms, st);
+  }
+  EpiPartialTMA::Params p;
+  if (!make_map_f32_3d(&p.map, part, g.N, g.M, g.split.splits, 32, 32)) return cudaErrorInvalidValue;
+  cudaError_t e = pair_gemm_bn<A_MN, B_MN, EpiPartialTMA>(bn, g, p, sms, st);
+  if (e != cudaSuccess) return e;
+  const long long sstride = (long long)g.M * g.N;
   return reduce_splits(part, g.split, sstride, g.M, g.N, alpha, out, ldo, transpose, reduce_name, st);
 }
 
@@ -621,11 +685,12 @@ dora_status_t bf16_norm(const dora_desc_t& d, const Plan& p, const void* W0, con
   ga.split = p.gram;
   ga.name = "gram_gemm";
   {
-    const long long sstride = (long long)r * r;
-    EpiPartialF32::Params pp{gram_part, r, sstride};
-    e = gemm_bn<false, false, EpiPartialF32>(bn_narrow_k(r), ga, pp, st);
+    EpiPartialTMA::Params pp;
+    if (!make_map_f32_3d(&pp.map, gram_part, r, r, p.gram.splits, 32, 32))
+      return gemm_status(cudaErrorInvalidValue, "dora_norm: Gram");
+    e = pair_gemm_bn<false, false, EpiPartialTMA>(p.gram_bn, ga, pp, p.sms, st);
     if (e != cudaSuccess) return gemm_status(e, "dora_norm: Gram");
-    const long long total = (long long)r * 2 * rp;
+    const long long total = (long long)r * 2 * (rp / 4);
     ProfRange pr("gram_finalize", st);
     e = launch_pdl(gram_finalize_kernel, dim3((unsigned)std::min<long long>(ceil_div(total, 256), 2048)), dim3(256),
                    0, st, (const float*)gram_part, p.gram.splits, r, rp, 0.5f * d.s, gs);
@@ -671,7 +736,7 @@ dora_status_t bf16_forward(const dora_desc_t& d, const Plan& p, int64_t T, const
   ua.N = r;
   ua.split = p.u;
   ua.name = "u_gemm";
-  cudaError_t e = narrow_gemm<false, false>(p.u_bn, ua, d.s, su, r, false, reinterpret_cast<float*>(ws + p.off_u_part),
+  cudaError_t e = narrow_gemm_pair<false, false>(p.u_bn, ua, d.s, su, r, false, reinterpret_cast<float*>(ws + p.off_u_part),
                                 "u_reduce", p.sms, st);
   if (e != cudaSuccess) return gemm_status(e, "dora_forward: LoRA down projection");
 
@@ -736,7 +801,7 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.N = r;
     a.split = p.du;
     a.name = "du_gemm";
-    cudaError_t e = narrow_gemm<false, true>(p.du_bn, a, d.s, du, r, false,
+    cudaError_t e = narrow_gemm_pair<false, true>(p.du_bn, a, d.s, du, r, false,
                                              reinterpret_cast<float*>(ws + p.off_du_part), "du_reduce", p.sms, st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: du");
   }
@@ -750,8 +815,8 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.N = r;
     a.split = p.dB;
     a.name = "dB_gemm";
-    cudaError_t e = narrow_gemm<true, true>(p.dB_bn, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dB), r, false,
-                                            reinterpret_cast<float*>(ws + p.off_dB_part), "dB_reduce", p.sms, st);
+    cudaError_t e = narrow_gemm_1cta<true, true>(p.dB_bn, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dB), r, false,
+                                                 reinterpret_cast<float*>(ws + p.off_dB_part), "dB_reduce", st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: dB");
   }
   // dA^T = x^T du, stored transposed into dA [r x d_in]
@@ -764,8 +829,8 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.N = r;
     a.split = p.dA;
     a.name = "dA_gemm";
-    cudaError_t e = narrow_gemm<true, true>(p.dA_bn, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dA), d_in, true,
-                                            reinterpret_cast<float*>(ws + p.off_dA_part), "dA_reduce", p.sms, st);
+    cudaError_t e = narrow_gemm_1cta<true, true>(p.dA_bn, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dA), d_in,
+                                                 true, reinterpret_cast<float*>(ws + p.off_dA_part), "dA_reduce", st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: dA");
   }
   // dx = [dz | du] [W0 ; A]  (W0 and A read MN-major: K rows, N = d_in contiguous)

@@ -23,6 +23,7 @@ struct Plan {
   int sms = 148;
   // norm
   Split gram, norm;
+  int gram_bn = 0;
   size_t off_gram_part = 0, off_gs = 0, off_norm_part = 0;
   // forward
   Split u;
@@ -48,6 +49,8 @@ inline int bn_narrow_k(int64_t r) {
   return r <= 16 ? 16 : r <= 32 ? 32 : r <= 64 ? 64 : r <= 128 ? 128 : r <= 256 ? 256 : r <= 384 ? 384 : 512;
 }
 inline int bn_narrow_mn(int64_t r) { return r <= 64 ? 64 : r <= 128 ? 128 : r <= 256 ? 256 : r <= 384 ? 384 : 512; }
+// Whole-rank tile width for CTA-pair GEMMs with K-major B (widths 64 .. 512).
+inline int bn_pair_k(int64_t r) { return r <= 64 ? 64 : r <= 128 ? 128 : r <= 256 ? 256 : r <= 384 ? 384 : 512; }
 
 int device_sm_count();
 Plan make_plan(const dora_desc_t& d, int64_t T, int op);

@@ -531,19 +531,32 @@ struct PairCfg {
 };
 
 // Work items are (output tile, K split) pairs: item = tile * splits + split.
+// Shared memory of a pair kernel: the stage ring, the epilogue's own staging
+// area (Epi::kStageOutBytes, if any), then the barriers.
+template <class Cfg, class Epi>
+struct PairLayout {
+  static constexpr int EPI_BYTES = Epi::kStageOutBytes;
+  static constexpr int STAGES_RAW = (kSmemBudget - EPI_BYTES) / Cfg::STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static_assert(STAGES >= 2, "stages");
+  static constexpr int SMEM_BYTES = STAGES * Cfg::STAGE_BYTES + EPI_BYTES + Cfg::BAR_BYTES + 1024;
+};
+
 template <class Cfg, class Epi>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_sm100_pair_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tA1,
                            const __grid_constant__ CUtensorMap tB0, const __grid_constant__ CUtensorMap tB1,
-                           const GemmGeom geom, const typename Epi::Params ep) {
+                           const GemmGeom geom, const __grid_constant__ typename Epi::Params ep) {
   static_assert(!Epi::kReadsA, "pair epilogues do not read A stages");
-  constexpr int STAGES = Cfg::STAGES;
+  constexpr int STAGES = PairLayout<Cfg, Epi>::STAGES;
+  constexpr int EPI_BYTES = PairLayout<Cfg, Epi>::EPI_BYTES;
   constexpr int NACC = Cfg::NUM_ACC;
   constexpr uint32_t ACC_COLS = Cfg::ACC_COLS;
   constexpr uint32_t TMEM_COLS = Cfg::TMEM_COLS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint8_t* epi_smem = smem + STAGES * Cfg::STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi_smem + EPI_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* accf = empty + STAGES;  // [2]
   uint64_t* acce = accf + 2;        // [2], used in the leader only
@@ -716,8 +729,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       c.n0 = tn * Cfg::BN;
       c.split = split;
       c.has_acc = min(kb_total, kb_begin + kps) > kb_begin;
-      c.stage_smem = nullptr;
-      c.stage_bytes = 0;
+      c.stage_smem = epi_smem;
+      c.stage_bytes = EPI_BYTES;
       c.aux_bar = nullptr;
       c.tA1 = &tA1;
       c.tile_id = t;
@@ -760,6 +773,7 @@ struct EpiStoreBF16 {
   };
   using RowState = NoRowState;
   static constexpr bool kReadsA = false;
+  static constexpr int kStageOutBytes = 0;
   __device__ static void on_a_stage(const Params&, RowState&, const uint8_t*, bool) {}
   template <int BN>
   __device__ static void run(const Params& p, RowState&, const EpiCtx& c, const GemmGeom& g) {
@@ -794,6 +808,7 @@ struct EpiPartialF32 {
   };
   using RowState = NoRowState;
   static constexpr bool kReadsA = false;
+  static constexpr int kStageOutBytes = 0;
   __device__ static void on_a_stage(const Params&, RowState&, const uint8_t*, bool) {}
   template <int BN>
   __device__ static void run(const Params& p, RowState&, const EpiCtx& c, const GemmGeom& g) {
@@ -807,6 +822,49 @@ struct EpiPartialF32 {
         if (col + 4 * j < BN && n + 4 * j < g.N)
           *reinterpret_cast<float4*>(base + n + 4 * j) = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
     });
+  }
+};
+
+// fp32 partial tiles written by TMA: each epilogue warp stages its 32 rows x
+// 32 columns (128 bytes per row, 128-byte swizzle) in one of two 4 KB buffers
+// of its own and stores them with a 3-D bulk tensor store over
+// [split][row][column], which clips rows past M and columns past N.
+struct EpiPartialTMA {
+  struct Params {
+    CUtensorMap map;  // fp32 {N, M, splits}, box {32, 32, 1}, 128-byte swizzle
+  };
+  using RowState = NoRowState;
+  static constexpr bool kReadsA = false;
+  static constexpr int kStageOutBytes = 4 * 2 * 4096;
+  __device__ static void on_a_stage(const Params&, RowState&, const uint8_t*, bool) {}
+  template <int BN>
+  __device__ static void run(const Params& p, RowState&, const EpiCtx& c, const GemmGeom& g) {
+    static_assert(BN % 32 == 0, "whole 32-column chunks");
+    const int q = c.row >> 5;
+    const int lane = c.row & 31;
+    uint8_t* bufs = c.stage_smem + q * 8192;
+    const int row0 = c.m - lane;
+    int chunk = 0;
+    for_each_acc_chunk<BN>(c, [&](int col, float* v) {
+      uint8_t* buf = bufs + (chunk & 1) * 4096;
+      if (chunk >= 2) {
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<float4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+            make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && c.n0 + col < g.N && row0 < g.M) {
+        tma_store_3d(&p.map, buf, c.n0 + col, row0, c.split);
+        bulk_commit();
+      }
+      ++chunk;
+    });
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 };
 
