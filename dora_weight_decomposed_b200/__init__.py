@@ -10,6 +10,7 @@ every call raises.
     norm, g, gm1 = dora_norm(W0, A, B, m, s)
     y, su, pre   = dora_forward(x, W0, A, B, gm1, s)
     dm, dA, dB, dx = dora_backward(dy, x, W0, A, B, norm, g, su, pre, s)
+    W_merged     = dora_merge(W0, A, B, g, s)
 
 bf16 tensors use the tcgen05 tensor-core path; fp32 tensors use the SIMT path.
 """
@@ -20,17 +21,18 @@ import os
 import threading
 
 __all__ = ["DoraError", "load_library", "library_path", "dora_workspace_size", "dora_norm", "dora_forward",
-           "dora_norm_noalloc", "dora_backward", "dora_device_status", "dora_last_error", "dora_version",
+           "dora_norm_noalloc", "dora_backward", "dora_merge", "dora_device_status", "dora_last_error",
+           "dora_version",
            "dora_profile_start",
            "dora_profile_stop", "dora_profile_count", "dora_profile_read", "DORA_OP_NORM",
            "DORA_OP_FORWARD", "DORA_OP_BACKWARD", "STATUS_NAMES", "EXPORTED_SYMBOLS"]
 
 DORA_BF16, DORA_FP32 = 0, 1
-DORA_OP_NORM, DORA_OP_FORWARD, DORA_OP_BACKWARD = 0, 1, 2
+DORA_OP_NORM, DORA_OP_FORWARD, DORA_OP_BACKWARD, DORA_OP_MERGE = 0, 1, 2, 3
 STATUS_NAMES = {0: "DORA_OK", 1: "DORA_EINVAL", 2: "DORA_EUNSUPPORTED", 3: "DORA_EWORKSPACE", 4: "DORA_ECUDA",
                 5: "DORA_ETIMEOUT"}
 EXPORTED_SYMBOLS = ("dora_workspace_size", "dora_norm", "dora_norm_noalloc", "dora_forward", "dora_backward",
-                    "dora_device_status",
+                    "dora_merge", "dora_device_status",
                     "dora_profile_start", "dora_profile_stop", "dora_profile_count", "dora_profile_read",
                     "dora_last_error", "dora_version")
 
@@ -80,6 +82,8 @@ def load_library() -> ctypes.CDLL:
         lib.dora_forward.restype = ctypes.c_int
         lib.dora_backward.argtypes = [DP, I64, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
         lib.dora_backward.restype = ctypes.c_int
+        lib.dora_merge.argtypes = [DP, P, P, P, P, P, P, SZ, P]
+        lib.dora_merge.restype = ctypes.c_int
         lib.dora_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint)]
         lib.dora_device_status.restype = ctypes.c_int
         lib.dora_profile_start.argtypes = [ctypes.c_int]
@@ -238,6 +242,23 @@ def dora_backward(dy, x, W0, A, B, norm, g, su_save, pre_save, s: float, *, need
                              _ptr(g), _ptr(su_save), _ptr(pre_save), _ptr(dm), _ptr(dA), _ptr(dB), _ptr(dx),
                              _ptr(wsb), nbytes, _stream_ptr(stream)))
     return dm, dA, dB, dx
+
+
+def dora_merge(W0, A, B, g, s: float, *, out=None, ws=None, stream=None):
+    """Merged weight diag(g) (W0 + s B A) for deployment; out may be W0 (in place)."""
+    torch = _torch()
+    lib = load_library()
+    d_out, d_in = W0.shape
+    r = A.shape[0]
+    _shape(A, (r, d_in), "A")
+    _shape(B, (d_out, r), "B")
+    _shape(g, (d_out,), "g")
+    desc = _desc(d_out, d_in, r, W0.dtype, s)
+    out = torch.empty_like(W0) if out is None else out
+    wsb, nbytes = _workspace(desc, 0, DORA_OP_MERGE, W0.device, ws)
+    _check(lib.dora_merge(ctypes.byref(desc), _ptr(W0), _ptr(A), _ptr(B), _ptr(g), _ptr(out), _ptr(wsb), nbytes,
+                          _stream_ptr(stream)))
+    return out
 
 
 def dora_device_status(stream=None) -> int:

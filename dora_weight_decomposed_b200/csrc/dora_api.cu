@@ -290,8 +290,24 @@ using namespace dora;
 extern "C" {
 
 size_t dora_workspace_size(const dora_desc_t* desc, int64_t T, int op) {
-  if (!check_desc(desc) || !check_T(T) || op < DORA_OP_NORM || op > DORA_OP_BACKWARD) return 0;
+  if (!check_desc(desc) || !check_T(T) || op < DORA_OP_NORM || op > DORA_OP_MERGE) return 0;
   return make_plan(*desc, T, op).total;
+}
+
+dora_status_t dora_merge(const dora_desc_t* desc, const void* W0, const void* A, const void* B, const float* g,
+                         void* W_out, void* ws, size_t ws_bytes, dora_stream_t stream) {
+  if (!check_desc(desc)) return DORA_EINVAL;
+  const size_t al = tensor_align(desc);
+  if (!check_ptr(W0, "W0", al) || !check_ptr(A, "A", al) || !check_ptr(B, "B", al) || !check_ptr(g, "g", 4) ||
+      !check_ptr(W_out, "W_out", al))
+    return DORA_EINVAL;
+  const Plan p = make_plan(*desc, 0, DORA_OP_MERGE);
+  dora_status_t s = check_ws(p, ws, ws_bytes);
+  if (s != DORA_OK) return s;
+  if ((s = check_device(desc)) != DORA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (desc->dtype == DORA_BF16) return bf16_merge(*desc, p, W0, A, B, g, W_out, reinterpret_cast<uint8_t*>(ws), st);
+  return f32_merge(*desc, (const float*)W0, (const float*)A, (const float*)B, g, (float*)W_out, st);
 }
 
 dora_status_t dora_norm(const dora_desc_t* desc, const void* W0, const void* A, const void* B, const float* m,

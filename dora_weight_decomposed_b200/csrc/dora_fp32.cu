@@ -150,6 +150,29 @@ __global__ void f32_dm_finalize_kernel(const float* __restrict__ part, int npart
   dm[i] = s / C[i];
 }
 
+// W_out[i][j] = g_i (W0[i][j] + s sum_k B[i][k] A[k][j]); one thread per element.
+__global__ void f32_merge_kernel(const float* __restrict__ W0, const float* __restrict__ A,
+                                 const float* __restrict__ B, const float* __restrict__ g, float* W_out, int d_out,
+                                 int d_in, int r, float s) {
+  const long long total = (long long)d_out * d_in;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int i = (int)(e / d_in), j = (int)(e % d_in);
+    float acc = 0.f;
+    for (int k = 0; k < r; ++k) acc = fmaf(B[(long long)i * r + k], A[(long long)k * d_in + j], acc);
+    W_out[e] = g[i] * fmaf(s, acc, W0[e]);
+  }
+}
+
+dora_status_t f32_merge(const dora_desc_t& d, const float* W0, const float* A, const float* B, const float* g,
+                        float* W_out, cudaStream_t st) {
+  const long long total = d.d_out * d.d_in;
+  ProfRange pr("f32_merge", st);
+  f32_merge_kernel<<<(unsigned)std::min<long long>(cdiv(total, 256), 4096), 256, 0, st>>>(
+      W0, A, B, g, W_out, (int)d.d_out, (int)d.d_in, (int)d.r, d.s);
+  return cuda_status(cudaGetLastError(), "dora_merge (fp32)");
+}
+
 dora_status_t f32_norm(const dora_desc_t& d, const Plan& p, const float* W0, const float* A, const float* B,
                        const float* m, float* C, float* g, float* gm1, uint8_t* ws, cudaStream_t st) {
   const int r = (int)d.r, d_in = (int)d.d_in, d_out = (int)d.d_out;

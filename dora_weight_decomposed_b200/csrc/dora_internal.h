@@ -72,6 +72,9 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
                             const void* su, const void* pre, float* dm, void* dA, void* dB, void* dx,
                             uint8_t* ws, cudaStream_t st);
 
+dora_status_t bf16_merge(const dora_desc_t& d, const Plan& p, const void* W0, const void* A, const void* B,
+                         const float* g, void* W_out, uint8_t* ws, cudaStream_t st);
+
 // fp32 path (SIMT kernels)
 dora_status_t f32_norm(const dora_desc_t& d, const Plan& p, const float* W0, const float* A, const float* B,
                        const float* m, float* C, float* g, float* gm1, uint8_t* ws, cudaStream_t st);
@@ -95,6 +98,9 @@ class ProfRange {
   cudaStream_t st_;
   int idx_;
 };
+
+dora_status_t f32_merge(const dora_desc_t& d, const float* W0, const float* A, const float* B, const float* g,
+                        float* W_out, cudaStream_t st);
 
 inline dora_status_t cuda_status(cudaError_t e, const char* where) {
   if (e == cudaSuccess) return DORA_OK;

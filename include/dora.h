@@ -60,7 +60,7 @@ typedef enum {
 
 typedef enum { DORA_BF16 = 0, DORA_FP32 = 1 } dora_dtype_t;
 
-typedef enum { DORA_OP_NORM = 0, DORA_OP_FORWARD = 1, DORA_OP_BACKWARD = 2 } dora_op_t;
+typedef enum { DORA_OP_NORM = 0, DORA_OP_FORWARD = 1, DORA_OP_BACKWARD = 2, DORA_OP_MERGE = 3 } dora_op_t;
 
 typedef struct {
   int64_t d_out;      /* output features (rows of W0, B, entries of m)   */
@@ -149,6 +149,19 @@ DORA_API dora_status_t dora_backward(const dora_desc_t* desc, int64_t T, const v
                             const void* A, const void* B, const float* norm, const float* g, const void* su_save,
                             const void* pre_save, float* dm, void* dA, void* dB, void* dx, void* ws,
                             size_t ws_bytes, dora_stream_t stream);
+
+/*
+ * dora_merge -- the merged deployment weight W' = diag(g) (W0 + s B A).
+ *
+ * DoRA notes Algorithm 1 steps 16-17 (merge after training: m (W0 + BA) / C
+ * stored as one dense weight, so inference costs a plain linear layer).
+ * In:  W0 [d_out x d_in], A [r x d_in], B [d_out x r] (dtype); g [d_out] fp32
+ *      from dora_norm. Out: W_out [d_out x d_in] (dtype), rounded once.
+ * W_out may be W0 itself (in-place merge): each output element is written by
+ * the thread that read its W0 value, and nothing else reads W0.
+ */
+DORA_API dora_status_t dora_merge(const dora_desc_t* desc, const void* W0, const void* A, const void* B,
+                                  const float* g, void* W_out, void* ws, size_t ws_bytes, dora_stream_t stream);
 
 /*
  * dora_device_status -- synchronise `stream`, then read and clear the library's

@@ -6,6 +6,7 @@ Tolerances (per output tensor):
   g - 1                 max |gpu - ref| <= 1e-3 * max |ref| (near-unity check)
   bf16 y, dm, dA, dB, dx  ||gpu - ref||_F / ||ref||_F <= 2e-2 and cosine >= 0.9999
   fp32 y, dm, dA, dB, dx  ||gpu - ref||_F / ||ref||_F <= 1e-4 and cosine >= 0.9999
+  merged weight         element-wise, in tests/test_merge_gpu.py
 """
 from __future__ import annotations
 

@@ -123,3 +123,18 @@ def test_workspace_checks(lib):
 
 def test_device_status_rejects_null(lib):
     assert lib.dora_device_status(None, None) == 1
+
+
+def test_merge_validation(lib):
+    d = _desc()
+    fake = ctypes.c_void_p(4096)
+    # The merge needs no workspace.
+    assert lib.dora_workspace_size(ctypes.byref(d), 0, 3) == 0
+    assert lib.dora_workspace_size(ctypes.byref(d), 0, 4) == 0
+    st = lib.dora_merge(ctypes.byref(d), fake, fake, fake, fake, None, None, 0, None)
+    assert st == 1 and "W_out" in dw.dora_last_error()
+    st = lib.dora_merge(ctypes.byref(d), fake, fake, ctypes.c_void_p(4096 + 8), fake, fake, None, 0, None)
+    assert st == 1 and "aligned" in dw.dora_last_error()
+    bad = _desc(r=12)
+    st = lib.dora_merge(ctypes.byref(bad), fake, fake, fake, fake, fake, None, 0, None)
+    assert st == 1
