@@ -25,7 +25,6 @@ from __future__ import annotations
 import argparse
 import datetime
 import hashlib
-import glob
 import json
 import os
 import statistics
@@ -58,6 +57,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=256, help="tokens per reference-arm step")
     ap.add_argument("--ref-rows", type=int, default=1024, help="output rows per reference-arm step")
+    ap.add_argument("--no-merge", action="store_true",
+                    help="skip the cached-norm inference and deployment-merge measurements")
     return ap.parse_args(argv)
 
 
@@ -87,29 +88,46 @@ def kernel_work(name, wl):
         "dB_gemm": (2 * T * do * r, b * (T * do + T * r + do * r)),
         "dA_gemm": (2 * T * di * r, b * (T * di + T * r + r * di)),
         "dx_gemm": (2 * T * di * (do + r), b * (T * do + do * di + T * r + r * di + T * di)),
+        "merge_gemm": (2 * do * di * r + 3 * do * di, b * (2 * do * di + do * r + r * di) + 4 * do),
     }
     return table.get(name, (0, 0))
 
 
-def source_hash():
+# Source files that define each kernel: DRAM traffic recorded by ncu stays
+# valid only while these files are unchanged.
+KERNEL_SOURCES = {
+    "fwd_compose_gemm": ("sm100_ptx.cuh", "gemm_sm100.cuh", "dora_bf16.cu"),
+    "merge_gemm": ("sm100_ptx.cuh", "gemm_sm100.cuh", "merge_sm100.cuh", "dora_bf16.cu"),
+}
+
+
+def source_hash(kernel):
+    names = KERNEL_SOURCES.get(kernel)
+    if names is None:
+        return None
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "dora_weight_decomposed_b200", "csrc", "*"))):
-        with open(p, "rb") as f:
+    for n in names:
+        with open(os.path.join(ROOT, "dora_weight_decomposed_b200", "csrc", n), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel):
-    """DRAM bytes per launch from the committed ncu summary, if taken on the current sources."""
-    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
-    if not os.path.exists(path):
+    """DRAM bytes per launch from the committed ncu summary (profiles/ncu_traffic.md),
+    if it was taken on the kernel's current sources; else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.md")
+    want = source_hash(kernel)
+    if want is None or not os.path.exists(path):
         return None
     with open(path) as f:
-        d = json.load(f)
-    if d.get("source_hash") != source_hash():
-        return None
-    k = d.get("kernels", {}).get(kernel)
-    return None if k is None else k.get("dram_bytes_per_launch")
+        for line in f:
+            cells = [c.strip() for c in line.strip().strip("|").split("|")]
+            if len(cells) >= 3 and cells[0] == kernel and cells[1] == want:
+                try:
+                    return float(cells[2])
+                except ValueError:
+                    return None
+    return None
 
 
 # ---------------------------------------------------------------- clocks
@@ -460,6 +478,63 @@ def run_ours(args, wl, cfg):
         e2e = {"value": world * T * len(evs) / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": len(evs), "api": "dora_norm/dora_forward/dora_backward (eager)"}
 
+    # ---- cached-norm inference: forward only, norm reused, nothing saved for a backward
+    infer = None
+    if rank == 0 and not args.no_merge:
+        wsi = torch.empty(max(dw.dora_workspace_size(do, di, r, bf, s, T, dw.DORA_OP_FORWARD), 256),
+                          dtype=torch.uint8, device=dev)
+        call_inf = lambda: dw.dora_forward(x, W0, A, B, gm1, s, y=y, save_for_backward=False, ws=wsi)
+        call_inf()
+        gi = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gi):
+            call_inf()
+        iev = []
+        for i in range(max(3, args.warmup) + 20):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            gi.replay()
+            e1.record()
+            if i >= max(3, args.warmup):
+                iev.append((e0, e1))
+        torch.cuda.synchronize()
+        i_ms = statistics.median(a.elapsed_time(b_) for a, b_ in iev)
+        fl = 2 * T * do * (di + r) + 2 * T * di * r
+        infer = {"value": T / (i_ms * 1e-3), "unit": UNIT, "ms_per_batch": i_ms, "tflops": fl / (i_ms * 1e-3) / 1e12,
+                 "calls": len(iev), "api": "dora_forward(save_for_backward=False) with the norm of a prior dora_norm",
+                 "l2": "flushed before every call"}
+        del gi, wsi
+
+    # ---- deployment merge W' = diag(g) (W0 + s B A) on the same layer (not part of the step)
+    merge = None
+    if rank == 0 and not args.no_merge:
+        Wm = torch.empty_like(W0)
+        call_merge = lambda: dw.dora_merge(W0, A, B, g, s, out=Wm)
+        for _ in range(3):
+            call_merge()
+        mev = []
+        for _ in range(20):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            call_merge()
+            e1.record()
+            mev.append((e0, e1))
+        torch.cuda.synchronize()
+        m_ms = statistics.median(a.elapsed_time(b_) for a, b_ in mev)
+        fl, by = kernel_work("merge_gemm", wl)
+        gbs, tfl = by / (m_ms * 1e-3) / 1e9, fl / (m_ms * 1e-3) / 1e12
+        # Bound: the larger of HBM time and tensor time at the measured burst peaks.
+        hbm_bound = by / peaks["hbm_gbs"] >= fl / (peaks["bf16_tflops"] * 1e3)
+        mroof = ({"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s"} if hbm_bound else
+                 {"bound": "tensor", "achieved": tfl, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"})
+        mroof["frac"] = mroof["achieved"] / mroof["peak"]
+        mroof["peak_source"] = f"{peak_src} ({'hbm_gbs' if hbm_bound else 'bf16_tflops'}, burst)"
+        mroof["traffic"] = recorded_traffic("merge_gemm")
+        merge = {"us": m_ms * 1e3, "gbs": gbs, "tflops": tfl, "calls": len(mev), "roofline": mroof,
+                 "l2": "flushed before every call", "api": "dora_merge"}
+        del Wm
+
     status = dw.dora_device_status()
 
     cpu = None
@@ -478,7 +553,8 @@ def run_ours(args, wl, cfg):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
             "norm_tflops": norm_flops / (phase_ms["norm"] * 1e-3) / 1e12, "phase_ms": phase_ms,
-            "roofline": roof, "kernels": kernels, "gpu_launches": int(launches_per_step * args.steps),
+            "roofline": roof, "kernels": kernels, "inference": infer, "merge": merge,
+            "gpu_launches": int(launches_per_step * args.steps),
             "clocks": clocks.summary(), "e2e": e2e, "cpu_baseline": cpu, "device_status": status,
             "step_ms_min": min(step_ms), "step_ms_median": statistics.median(step_ms)}
     print(json.dumps(line), flush=True)

@@ -21,6 +21,7 @@
 
 #include "dora_internal.h"
 #include "gemm_sm100.cuh"
+#include "merge_sm100.cuh"
 
 namespace dora {
 
@@ -423,42 +424,6 @@ struct EpiCompose {
   }
 };
 
-// Merge: out[m, n] = g_m (W0[m, n] + s acc[m, n]) with acc = (B A)[m, n], bf16.
-// Each thread reads the W0 values of exactly the elements it writes.
-struct EpiMerge {
-  struct Params {
-    const __nv_bfloat16* W0;
-    __nv_bfloat16* out;
-    const float* g;
-    float s;
-    long long ld;
-  };
-  using RowState = NoRowState;
-  static constexpr bool kReadsA = false;
-  static constexpr int kStageOutBytes = 0;
-  __device__ static void on_a_stage(const Params&, RowState&, const uint8_t*, bool) {}
-  template <int BN>
-  __device__ static void run(const Params& p, RowState&, const EpiCtx& c, const GemmGeom& g) {
-    const bool row_ok = c.m < g.M;
-    const float gm = row_ok ? p.g[c.m] : 0.f;
-    for_each_acc_chunk<BN>(c, [&](int col, float* v) {
-      if (!row_ok) return;
-      const int n = c.n0 + col;
-      const long long off = (long long)c.m * p.ld + n;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (col + 8 * j < BN && n + 8 * j < g.N) {
-          float w[8], o[8];
-          unpack_bf16x8(*reinterpret_cast<const uint4*>(p.W0 + off + 8 * j), w);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) o[i] = gm * fmaf(p.s, v[8 * j + i], w[i]);
-          store_bf16x8(p.out + off + 8 * j, o);
-        }
-      }
-    });
-  }
-};
-
 template <int BN>
 static cudaError_t norm_gemm_bn(const GemmArgs& g, const EpiNorm::Params& ep, cudaStream_t st) {
   return launch_gemm<GemmCfg<BN, false, false>, EpiNorm>(g, ep, st);
@@ -795,22 +760,32 @@ dora_status_t bf16_forward(const dora_desc_t& d, const Plan& p, int64_t T, const
   return gemm_status(e, "dora_forward: base GEMM with compose");
 }
 
+template <class Cfg>
+static cudaError_t launch_merge(const CUtensorMap& ta, const CUtensorMap& tb, const MergeGeom& geom, long long pairs,
+                                cudaStream_t st) {
+  auto kern = merge_pair_kernel<Cfg>;
+  static std::atomic<unsigned long long> smem_set{0};
+  cudaError_t e = set_smem_once(smem_set, kern, Cfg::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  ProfRange pr("merge_gemm", st);
+  return launch_pdl(kern, dim3((unsigned)(2 * pairs)), dim3(Cfg::THREADS), (size_t)Cfg::SMEM_BYTES, st, ta, tb, geom);
+}
+
 dora_status_t bf16_merge(const dora_desc_t& d, const Plan& p, const void* W0, const void* A, const void* B,
                          const float* g, void* W_out, uint8_t*, cudaStream_t st) {
-  const int r = (int)d.r, d_in = (int)d.d_in, d_out = (int)d.d_out;
-  // acc = B A: A-operand B [d_out x r] (K = r contiguous), B-operand A [r x d_in] read MN-major.
-  GemmArgs a;
-  a.a0 = Mat{B, d_out, r, r};
-  a.b0 = Mat{A, r, d_in, d_in};
-  a.K0 = r;
-  a.M = d_out;
-  a.N = d_in;
-  a.split.splits = 1;
-  a.split.kb_per_split = (int)ceil_div(r, kBK);
-  a.name = "merge_gemm";
-  EpiMerge::Params mp{reinterpret_cast<const __nv_bfloat16*>(W0), reinterpret_cast<__nv_bfloat16*>(W_out), g, d.s,
-                      d_in};
-  cudaError_t e = launch_gemm_pair<PairCfg<256, false, true>, EpiMerge>(a, mp, p.sms, st);
+  // B A with A-operand = rows of B [d_out x r] (K = r contiguous) and
+  // B-operand = A [r x d_in] read MN-major; W0 is streamed by the epilogue.
+  CUtensorMap ta, tb;
+  t_detail.clear();
+  if (!make_map(&ta, Mat{B, d.d_out, d.r, d.r}, kBM, "B") || !make_map(&tb, Mat{A, d.r, d.d_in, d.d_in}, 64, "A"))
+    return gemm_status(cudaErrorInvalidValue, "dora_merge");
+  const int kb = (int)ceil_div(d.r, kBK);
+  const MergeGeom geom{(int)d.d_out, (int)d.d_in, kb, g, d.s, reinterpret_cast<const __nv_bfloat16*>(W0),
+                       reinterpret_cast<__nv_bfloat16*>(W_out)};
+  const long long items = ceil_div(d.d_out, 2 * kBM) * ceil_div(d.d_in, 256);
+  const long long pairs = std::max<long long>(1, std::min<long long>(items, p.sms / 2));
+  cudaError_t e = launch_merge<MergeCfg<4, 6>>(ta, tb, geom, pairs, st);
+  if (e == cudaSuccess) e = cudaGetLastError();
   return gemm_status(e, "dora_merge");
 }
 

@@ -225,9 +225,14 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Arrive once on an mbarrier given by its shared::cluster address (possibly in the peer CTA).
+// Arrive once on an mbarrier given by its shared::cluster address (possibly in
+// the peer CTA). Used to hand a TMEM accumulator back to the MMA issuer: the
+// thread's tcgen05.ld reads are already complete (tcgen05.wait::ld) and
+// fenced (tcgen05.fence::before_thread_sync), so the default CTA-scope
+// release is enough. A cluster-scope release would also wait for every
+// global store the thread still has in flight.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // 2-D tiled load into this CTA's shared memory whose completion is counted on
