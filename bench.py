@@ -58,7 +58,7 @@ def parse_args(argv=None):
     ap.add_argument("--ref-tokens", type=int, default=256, help="tokens per reference-arm step")
     ap.add_argument("--ref-rows", type=int, default=1024, help="output rows per reference-arm step")
     ap.add_argument("--no-merge", action="store_true",
-                    help="skip the cached-norm inference and deployment-merge measurements")
+                    help="skip the inference, full-gradient and deployment-merge measurements")
     return ap.parse_args(argv)
 
 
@@ -505,6 +505,32 @@ def run_ours(args, wl, cfg):
                  "l2": "flushed before every call"}
         del gi, wsi
 
+    # ---- the backward without the detach of the norm (appendix A eq. A.1), same layer and batch
+    full_bwd = None
+    if rank == 0 and not args.no_merge:
+        wsf = torch.empty(max(dw.dora_workspace_size(do, di, r, bf, s, T, dw.DORA_OP_BACKWARD_FULL), 256),
+                          dtype=torch.uint8, device=dev)
+        call_full = lambda: dw.dora_backward_full(dy, x, W0, A, B, C, g, su, pre, s, dm=dm, dA=dA, dB=dB, dx=dx,
+                                                  ws=wsf)
+        call_full()
+        gf = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gf):
+            call_full()
+        fev = []
+        for i in range(max(3, args.warmup) + 20):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            gf.replay()
+            e1.record()
+            if i >= max(3, args.warmup):
+                fev.append((e0, e1))
+        torch.cuda.synchronize()
+        f_ms = statistics.median(a.elapsed_time(b_) for a, b_ in fev)
+        full_bwd = {"ms": f_ms, "detached_ms": phase_ms["backward"], "calls": len(fev),
+                    "api": "dora_backward_full", "l2": "flushed before every call"}
+        del gf, wsf
+
     # ---- deployment merge W' = diag(g) (W0 + s B A) on the same layer (not part of the step)
     merge = None
     if rank == 0 and not args.no_merge:
@@ -553,7 +579,7 @@ def run_ours(args, wl, cfg):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
             "norm_tflops": norm_flops / (phase_ms["norm"] * 1e-3) / 1e12, "phase_ms": phase_ms,
-            "roofline": roof, "kernels": kernels, "inference": infer, "merge": merge,
+            "roofline": roof, "kernels": kernels, "inference": infer, "backward_full": full_bwd, "merge": merge,
             "gpu_launches": int(launches_per_step * args.steps),
             "clocks": clocks.summary(), "e2e": e2e, "cpu_baseline": cpu, "device_status": status,
             "step_ms_min": min(step_ms), "step_ms_median": statistics.median(step_ms)}

@@ -9,7 +9,7 @@ every call raises.
 
     norm, g, gm1 = dora_norm(W0, A, B, m, s)
     y, su, pre   = dora_forward(x, W0, A, B, gm1, s)
-    dm, dA, dB, dx = dora_backward(dy, x, W0, A, B, norm, g, su, pre, s)
+    dm, dA, dB, dx = dora_backward(dy, x, W0, A, B, norm, g, su, pre, s)    # full=True: no detach
     W_merged     = dora_merge(W0, A, B, g, s)
 
 bf16 tensors use the tcgen05 tensor-core path; fp32 tensors use the SIMT path.
@@ -21,18 +21,19 @@ import os
 import threading
 
 __all__ = ["DoraError", "load_library", "library_path", "dora_workspace_size", "dora_norm", "dora_forward",
-           "dora_norm_noalloc", "dora_backward", "dora_merge", "dora_device_status", "dora_last_error",
+           "dora_norm_noalloc", "dora_backward", "dora_backward_full", "dora_merge", "dora_device_status", "dora_last_error",
            "dora_version",
            "dora_profile_start",
            "dora_profile_stop", "dora_profile_count", "dora_profile_read", "DORA_OP_NORM",
-           "DORA_OP_FORWARD", "DORA_OP_BACKWARD", "STATUS_NAMES", "EXPORTED_SYMBOLS"]
+           "DORA_OP_FORWARD", "DORA_OP_BACKWARD", "DORA_OP_MERGE", "DORA_OP_BACKWARD_FULL", "STATUS_NAMES",
+           "EXPORTED_SYMBOLS"]
 
 DORA_BF16, DORA_FP32 = 0, 1
-DORA_OP_NORM, DORA_OP_FORWARD, DORA_OP_BACKWARD, DORA_OP_MERGE = 0, 1, 2, 3
+DORA_OP_NORM, DORA_OP_FORWARD, DORA_OP_BACKWARD, DORA_OP_MERGE, DORA_OP_BACKWARD_FULL = 0, 1, 2, 3, 4
 STATUS_NAMES = {0: "DORA_OK", 1: "DORA_EINVAL", 2: "DORA_EUNSUPPORTED", 3: "DORA_EWORKSPACE", 4: "DORA_ECUDA",
                 5: "DORA_ETIMEOUT"}
 EXPORTED_SYMBOLS = ("dora_workspace_size", "dora_norm", "dora_norm_noalloc", "dora_forward", "dora_backward",
-                    "dora_merge", "dora_device_status",
+                    "dora_backward_full", "dora_merge", "dora_device_status",
                     "dora_profile_start", "dora_profile_stop", "dora_profile_count", "dora_profile_read",
                     "dora_last_error", "dora_version")
 
@@ -82,6 +83,8 @@ def load_library() -> ctypes.CDLL:
         lib.dora_forward.restype = ctypes.c_int
         lib.dora_backward.argtypes = [DP, I64, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
         lib.dora_backward.restype = ctypes.c_int
+        lib.dora_backward_full.argtypes = lib.dora_backward.argtypes
+        lib.dora_backward_full.restype = ctypes.c_int
         lib.dora_merge.argtypes = [DP, P, P, P, P, P, P, SZ, P]
         lib.dora_merge.restype = ctypes.c_int
         lib.dora_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint)]
@@ -217,9 +220,13 @@ def dora_forward(x, W0, A, B, gm1, s: float, *, save_for_backward: bool = True, 
     return y, su_save, pre_save
 
 
-def dora_backward(dy, x, W0, A, B, norm, g, su_save, pre_save, s: float, *, need_dx: bool = True, dm=None,
-                  dA=None, dB=None, dx=None, ws=None, stream=None):
-    """Detached-norm gradients (dm, dA, dB, dx); dx is None when need_dx is False."""
+def dora_backward(dy, x, W0, A, B, norm, g, su_save, pre_save, s: float, *, need_dx: bool = True, full: bool = False,
+                  dm=None, dA=None, dB=None, dx=None, ws=None, stream=None):
+    """Gradients (dm, dA, dB, dx); dx is None when need_dx is False.
+
+    Detached norm by default (dora_backward); full=True keeps the gradient
+    through the norm (dora_backward_full), which changes dA and dB only.
+    """
     torch = _torch()
     lib = load_library()
     T, d_in = x.shape
@@ -237,10 +244,11 @@ def dora_backward(dy, x, W0, A, B, norm, g, su_save, pre_save, s: float, *, need
         dx = torch.empty(T, d_in, dtype=x.dtype, device=dev)
     if not need_dx:
         dx = None
-    wsb, nbytes = _workspace(desc, T, DORA_OP_BACKWARD, dev, ws)
-    _check(lib.dora_backward(ctypes.byref(desc), T, _ptr(dy), _ptr(x), _ptr(W0), _ptr(A), _ptr(B), _ptr(norm),
-                             _ptr(g), _ptr(su_save), _ptr(pre_save), _ptr(dm), _ptr(dA), _ptr(dB), _ptr(dx),
-                             _ptr(wsb), nbytes, _stream_ptr(stream)))
+    wsb, nbytes = _workspace(desc, T, DORA_OP_BACKWARD_FULL if full else DORA_OP_BACKWARD, dev, ws)
+    fn = lib.dora_backward_full if full else lib.dora_backward
+    _check(fn(ctypes.byref(desc), T, _ptr(dy), _ptr(x), _ptr(W0), _ptr(A), _ptr(B), _ptr(norm), _ptr(g),
+              _ptr(su_save), _ptr(pre_save), _ptr(dm), _ptr(dA), _ptr(dB), _ptr(dx), _ptr(wsb), nbytes,
+              _stream_ptr(stream)))
     return dm, dA, dB, dx
 
 
@@ -319,3 +327,8 @@ def dora_norm_noalloc(W0, A, B, m, s: float, *, norm_out=None, g_out=None, gm1_o
     _check(fn(ctypes.byref(desc), _ptr(W0), _ptr(A), _ptr(B), _ptr(m), _ptr(norm_out), _ptr(g_out), _ptr(gm1_out),
               _stream_ptr(stream)))
     return norm_out, g_out, gm1_out
+
+
+def dora_backward_full(dy, x, W0, A, B, norm, g, su_save, pre_save, s: float, **kw):
+    """dora_backward with the gradient through the norm kept (appendix A eq. A.1)."""
+    return dora_backward(dy, x, W0, A, B, norm, g, su_save, pre_save, s, full=True, **kw)

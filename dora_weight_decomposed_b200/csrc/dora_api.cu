@@ -173,7 +173,7 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
       p.u = u.split;
       if (p.u.splits > 1) p.off_u_part = take((size_t)p.u.splits * T * r * 4);
       p.off_su = take((size_t)T * r * 2);
-    } else if (op == DORA_OP_BACKWARD && T > 0) {
+    } else if ((op == DORA_OP_BACKWARD || op == DORA_OP_BACKWARD_FULL) && T > 0) {
       p.off_dz = take((size_t)T * d_out * 2);
       p.dm_rowblocks = (int)cdiv(T, 256);
       p.off_dm_part = take((size_t)p.dm_rowblocks * d_out * 4);
@@ -193,6 +193,26 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
       // counters of the dm column strips, zeroed by one memset per call
       p.zero_bytes = (size_t)cdiv(d_out, 64) * 4;
       p.off_ctr = take(p.zero_bytes);
+      if (op == DORA_OP_BACKWARD_FULL) {
+        const int64_t rp = cdiv(r, 64) * 64;
+        p.off_kappa = take((size_t)d_out * 4);
+        p.off_bk = take((size_t)d_out * r * 2);
+        p.gram_bn = bn_pair_k(r);
+        const int64_t gram_max = std::max<int64_t>(1, (int64_t(8) << 20) / (r * r * 4));
+        p.gram = choose_split(cdiv(r, 256), cdiv(d_in, 64), p.sms / 2, kbB * (128 + p.gram_bn / 2.0), 0.0,
+                              (double)r * r, gram_max);
+        p.off_gram_part = take((size_t)p.gram.splits * r * r * 4);
+        p.off_gs = take((size_t)r * 2 * rp * 2);
+        const NarrowChoice q = choose_narrow(d_out, r, d_in + 2 * rp, false, p.sms);
+        p.q_bn = q.bn;
+        p.q = q.split;
+        p.off_q_part = take((size_t)p.q.splits * d_out * r * 4);
+        const NarrowChoice h = choose_narrow_1cta(r, r, d_out, true, p.sms);
+        p.h_bn = h.bn;
+        p.h = h.split;
+        if (p.h.splits > 1) p.off_h_part = take((size_t)p.h.splits * r * r * 4);
+        p.off_h = take((size_t)r * r * 2);
+      }
     }
   } else {
     if (op == DORA_OP_NORM) {
@@ -202,10 +222,17 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
     } else if (op == DORA_OP_FORWARD && T > 0) {
       p.off_f32_a = take((size_t)T * r * 4);
       p.off_f32_b = take((size_t)T * d_out * 4);
-    } else if (op == DORA_OP_BACKWARD && T > 0) {
+    } else if ((op == DORA_OP_BACKWARD || op == DORA_OP_BACKWARD_FULL) && T > 0) {
       p.off_f32_a = take((size_t)T * d_out * 4);
       p.off_f32_b = take((size_t)cdiv(T, 64) * d_out * 4);
       p.off_f32_c = take((size_t)T * r * 4);
+      if (op == DORA_OP_BACKWARD_FULL) {
+        p.off_kappa = take((size_t)d_out * 4);
+        p.off_bk = take((size_t)d_out * r * 4);
+        p.off_gs = take((size_t)r * r * 4);
+        p.off_q_part = take((size_t)d_out * r * 4);
+        p.off_h = take((size_t)r * r * 4);
+      }
     }
   }
   p.total = off;
@@ -290,7 +317,7 @@ using namespace dora;
 extern "C" {
 
 size_t dora_workspace_size(const dora_desc_t* desc, int64_t T, int op) {
-  if (!check_desc(desc) || !check_T(T) || op < DORA_OP_NORM || op > DORA_OP_MERGE) return 0;
+  if (!check_desc(desc) || !check_T(T) || op < DORA_OP_NORM || op > DORA_OP_BACKWARD_FULL) return 0;
   return make_plan(*desc, T, op).total;
 }
 
@@ -350,10 +377,10 @@ dora_status_t dora_forward(const dora_desc_t* desc, int64_t T, const void* x, co
                      (float*)y, (float*)su_save, (float*)pre_save, w, st);
 }
 
-dora_status_t dora_backward(const dora_desc_t* desc, int64_t T, const void* dy, const void* x, const void* W0,
-                            const void* A, const void* B, const float* norm, const float* g, const void* su_save,
-                            const void* pre_save, float* dm, void* dA, void* dB, void* dx, void* ws,
-                            size_t ws_bytes, dora_stream_t stream) {
+static dora_status_t backward_impl(bool full, const dora_desc_t* desc, int64_t T, const void* dy, const void* x,
+                                   const void* W0, const void* A, const void* B, const float* norm, const float* g,
+                                   const void* su_save, const void* pre_save, float* dm, void* dA, void* dB,
+                                   void* dx, void* ws, size_t ws_bytes, dora_stream_t stream) {
   if (!check_desc(desc) || !check_T(T)) return DORA_EINVAL;
   const size_t al = tensor_align(desc);
   // Per-token tensors have no elements when T == 0 and may then be NULL.
@@ -364,17 +391,35 @@ dora_status_t dora_backward(const dora_desc_t* desc, int64_t T, const void* dy, 
       !check_ptr(dm, "dm", 4) || !check_ptr(dA, "dA", al) || !check_ptr(dB, "dB", al) ||
       !check_opt_ptr(dx, "dx", al))
     return DORA_EINVAL;
-  const Plan p = make_plan(*desc, T, DORA_OP_BACKWARD);
+  const Plan p = make_plan(*desc, T, full ? DORA_OP_BACKWARD_FULL : DORA_OP_BACKWARD);
   dora_status_t s = check_ws(p, ws, ws_bytes);
   if (s != DORA_OK) return s;
   if ((s = check_device(desc)) != DORA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* w = reinterpret_cast<uint8_t*>(ws);
   if (desc->dtype == DORA_BF16)
-    return bf16_backward(*desc, p, T, dy, x, W0, A, B, norm, g, su_save, pre_save, dm, dA, dB, dx, w, st);
-  return f32_backward(*desc, p, T, (const float*)dy, (const float*)x, (const float*)W0, (const float*)A,
-                      (const float*)B, norm, g, (const float*)su_save, (const float*)pre_save, dm, (float*)dA,
-                      (float*)dB, (float*)dx, w, st);
+    return (full ? bf16_backward_full : bf16_backward)(*desc, p, T, dy, x, W0, A, B, norm, g, su_save, pre_save, dm,
+                                                       dA, dB, dx, w, st);
+  return (full ? f32_backward_full : f32_backward)(*desc, p, T, (const float*)dy, (const float*)x, (const float*)W0,
+                                                   (const float*)A, (const float*)B, norm, g, (const float*)su_save,
+                                                   (const float*)pre_save, dm, (float*)dA, (float*)dB, (float*)dx,
+                                                   w, st);
+}
+
+dora_status_t dora_backward(const dora_desc_t* desc, int64_t T, const void* dy, const void* x, const void* W0,
+                            const void* A, const void* B, const float* norm, const float* g, const void* su_save,
+                            const void* pre_save, float* dm, void* dA, void* dB, void* dx, void* ws,
+                            size_t ws_bytes, dora_stream_t stream) {
+  return backward_impl(false, desc, T, dy, x, W0, A, B, norm, g, su_save, pre_save, dm, dA, dB, dx, ws, ws_bytes,
+                       stream);
+}
+
+dora_status_t dora_backward_full(const dora_desc_t* desc, int64_t T, const void* dy, const void* x, const void* W0,
+                                 const void* A, const void* B, const float* norm, const float* g,
+                                 const void* su_save, const void* pre_save, float* dm, void* dA, void* dB, void* dx,
+                                 void* ws, size_t ws_bytes, dora_stream_t stream) {
+  return backward_impl(true, desc, T, dy, x, W0, A, B, norm, g, su_save, pre_save, dm, dA, dB, dx, ws, ws_bytes,
+                       stream);
 }
 
 dora_status_t dora_device_status(dora_stream_t stream, unsigned int* flags_out) {

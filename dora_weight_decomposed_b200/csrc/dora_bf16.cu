@@ -424,6 +424,40 @@ struct EpiCompose {
   }
 };
 
+// out[m][n] = out[m][n] + alpha acc[m][n]: the old bf16 value is read and the
+// sum rounded once. Each thread reads exactly the elements it writes.
+struct EpiAxpyBF16 {
+  struct Params {
+    __nv_bfloat16* out;
+    long long ldo;
+    float alpha;
+  };
+  using RowState = NoRowState;
+  static constexpr bool kReadsA = false;
+  static constexpr int kStageOutBytes = 0;
+  __device__ static void on_a_stage(const Params&, RowState&, const uint8_t*, bool) {}
+  template <int BN>
+  __device__ static void run(const Params& p, RowState&, const EpiCtx& c, const GemmGeom& g) {
+    const bool row_ok = c.m < g.M;
+    // for_each_acc_chunk is warp-collective: rows past M skip only the memory work.
+    for_each_acc_chunk<BN>(c, [&](int col, float* v) {
+      if (!row_ok) return;
+      const int n = c.n0 + col;
+      __nv_bfloat16* dst = p.out + (long long)c.m * p.ldo + n;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (col + 8 * j < BN && n + 8 * j < g.N) {
+          float o[8];
+          unpack_bf16x8(*reinterpret_cast<const uint4*>(dst + 8 * j), o);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) o[i] = fmaf(p.alpha, v[8 * j + i], o[i]);
+          store_bf16x8(dst + 8 * j, o);
+        }
+      }
+    });
+  }
+};
+
 template <int BN>
 static cudaError_t norm_gemm_bn(const GemmArgs& g, const EpiNorm::Params& ep, cudaStream_t st) {
   return launch_gemm<GemmCfg<BN, false, false>, EpiNorm>(g, ep, st);
@@ -482,11 +516,11 @@ __global__ void reduce_splits_bf16_kernel(const float* __restrict__ part, int sp
   }
 }
 
-// Gram finalize: x = (s/2) sum_z part[z] in fp32 (split order fixed), written
+// Gram finalize: x = scale sum_z part[z] in fp32 (split order fixed), written
 // as two bf16 halves Gs2[n] = [hi(x_n,0..r-1), 0 .. | lo(x_n,0..r-1), 0 ..]
 // with rp columns each, hi = bf16(x) and lo = bf16(x - hi), so hi + lo carries
 // x to about 2^-17. Each thread takes 4 consecutive columns of one half-row.
-__global__ void gram_finalize_kernel(const float* __restrict__ part, int splits, int r, int rp, float half_s,
+__global__ void gram_finalize_kernel(const float* __restrict__ part, int splits, int r, int rp, float scale,
                                      __nv_bfloat16* __restrict__ gs2) {
   pdl_trigger();
   pdl_wait();
@@ -510,7 +544,7 @@ __global__ void gram_finalize_kernel(const float* __restrict__ part, int splits,
         x.w += v.w;
       }
     }
-    const float xs[4] = {half_s * x.x, half_s * x.y, half_s * x.z, half_s * x.w};
+    const float xs[4] = {scale * x.x, scale * x.y, scale * x.z, scale * x.w};
     __nv_bfloat16 o[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -602,6 +636,55 @@ __global__ void __launch_bounds__(256) compose_bwd_bf16_kernel(const __nv_bfloat
   }
 }
 
+// Full gradient, per row n: kappa_n = g_n dm_n / C_n and Bk[n] = bf16(kappa_n B[n]).
+// One thread per 8 columns of a row; the row's first thread also stores kappa_n.
+__global__ void full_kappa_kernel(const float* __restrict__ g, const float* __restrict__ dm,
+                                  const float* __restrict__ C, const __nv_bfloat16* __restrict__ B, int d_out, int r,
+                                  float* __restrict__ kappa, __nv_bfloat16* __restrict__ Bk) {
+  pdl_trigger();
+  pdl_wait();
+  const int q = r / 8;
+  const long long total = (long long)d_out * q;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int n = (int)(i / q), c = (int)(i % q) * 8;
+    const float k = g[n] * dm[n] / C[n];
+    if (c == 0) kappa[n] = k;
+    float b[8];
+    unpack_bf16x8(*reinterpret_cast<const uint4*>(B + (long long)n * r + c), b);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) b[j] *= k;
+    store_bf16x8(Bk + (long long)n * r + c, b);
+  }
+}
+
+// Full gradient, dB[n][c] -= s kappa_n Q[n][c] with Q = sum_z part[z] (split
+// order fixed); the old bf16 dB is read and the result rounded once.
+__global__ void full_dB_kernel(const float* __restrict__ part, int splits, long long split_stride, int d_out, int r,
+                               const float* __restrict__ kappa, float s, __nv_bfloat16* __restrict__ dB) {
+  pdl_trigger();
+  pdl_wait();
+  const int q = r / 4;
+  const long long total = (long long)d_out * q;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int n = (int)(i / q), c = (int)(i % q) * 4;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int z = 0; z < splits; ++z) {
+      const float4 v = *reinterpret_cast<const float4*>(part + z * split_stride + (long long)n * r + c);
+      a.x += v.x;
+      a.y += v.y;
+      a.z += v.z;
+      a.w += v.w;
+    }
+    const float f = -s * kappa[n];
+    __nv_bfloat162* d2 = reinterpret_cast<__nv_bfloat162*>(dB + (long long)n * r + c);
+    const float2 o0 = __bfloat1622float2(d2[0]), o1 = __bfloat1622float2(d2[1]);
+    d2[0] = __floats2bfloat162_rn(fmaf(f, a.x, o0.x), fmaf(f, a.y, o0.y));
+    d2[1] = __floats2bfloat162_rn(fmaf(f, a.z, o1.x), fmaf(f, a.w, o1.y));
+  }
+}
+
 static cudaError_t reduce_splits(const float* part, const Split& sp, long long split_stride, int M, int N,
                                  float alpha, __nv_bfloat16* out, long long ldo, bool transpose, const char* name,
                                  cudaStream_t st) {
@@ -664,6 +747,31 @@ static cudaError_t narrow_gemm_pair(int bn, const GemmArgs& g, float alpha, __nv
 
 // ============================================================== operations
 
+// Gram G = A A^T (CTA pairs, split K into fp32 partials), then scale * G as
+// bf16 hi and lo halves [r x 2 rp] for a K-extension of a later GEMM.
+static cudaError_t gram_hi_lo(const dora_desc_t& d, const Plan& p, const void* A, float scale, float* gram_part,
+                              __nv_bfloat16* gs, cudaStream_t st) {
+  const int r = (int)d.r, d_in = (int)d.d_in;
+  const int rp = (int)ceil_div(r, kBK) * kBK;
+  GemmArgs ga;
+  ga.a0 = Mat{A, r, d_in, d_in};
+  ga.b0 = ga.a0;
+  ga.K0 = d_in;
+  ga.M = r;
+  ga.N = r;
+  ga.split = p.gram;
+  ga.name = "gram_gemm";
+  EpiPartialTMA::Params pp;
+  if (!make_map_f32_3d(&pp.map, gram_part, r, r, p.gram.splits, 32, 32)) return cudaErrorInvalidValue;
+  cudaError_t e = pair_gemm_bn<false, false, EpiPartialTMA>(p.gram_bn, ga, pp, p.sms, st);
+  if (e != cudaSuccess) return e;
+  const long long total = (long long)r * 2 * (rp / 4);
+  ProfRange pr("gram_finalize", st);
+  e = launch_pdl(gram_finalize_kernel, dim3((unsigned)std::min<long long>(ceil_div(total, 256), 2048)), dim3(256), 0,
+                 st, (const float*)gram_part, p.gram.splits, r, rp, scale, gs);
+  return e == cudaSuccess ? cudaGetLastError() : e;
+}
+
 dora_status_t bf16_norm(const dora_desc_t& d, const Plan& p, const void* W0, const void* A, const void* B,
                         const float* m, float* C, float* g, float* gm1, uint8_t* ws, cudaStream_t st) {
   const int r = (int)d.r, d_in = (int)d.d_in, d_out = (int)d.d_out;
@@ -677,28 +785,8 @@ dora_status_t bf16_norm(const dora_desc_t& d, const Plan& p, const void* W0, con
 
   // Gram G = A A^T in fp32 partials, then (s/2) G as bf16 hi and lo halves.
   const int rp = (int)ceil_div(r, kBK) * kBK;
-  GemmArgs ga;
-  ga.a0 = Mat{A, r, d_in, d_in};
-  ga.b0 = ga.a0;
-  ga.K0 = d_in;
-  ga.M = r;
-  ga.N = r;
-  ga.split = p.gram;
-  ga.name = "gram_gemm";
-  {
-    EpiPartialTMA::Params pp;
-    if (!make_map_f32_3d(&pp.map, gram_part, r, r, p.gram.splits, 32, 32))
-      return gemm_status(cudaErrorInvalidValue, "dora_norm: Gram");
-    e = pair_gemm_bn<false, false, EpiPartialTMA>(p.gram_bn, ga, pp, p.sms, st);
-    if (e != cudaSuccess) return gemm_status(e, "dora_norm: Gram");
-    const long long total = (long long)r * 2 * (rp / 4);
-    ProfRange pr("gram_finalize", st);
-    e = launch_pdl(gram_finalize_kernel, dim3((unsigned)std::min<long long>(ceil_div(total, 256), 2048)), dim3(256),
-                   0, st, (const float*)gram_part, p.gram.splits, r, rp, 0.5f * d.s, gs);
-    if (e != cudaSuccess) return cuda_status(e, "dora_norm: Gram finalize");
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_status(e, "dora_norm: Gram finalize");
-  }
+  e = gram_hi_lo(d, p, A, 0.5f * d.s, gram_part, gs, st);
+  if (e != cudaSuccess) return gemm_status(e, "dora_norm: Gram");
 
   // acc = [W0 | B | B] [A | Gs_hi | Gs_lo]^T with the factored-norm epilogue,
   // finished (C, g, g - 1) by the last split of each row tile.
@@ -880,6 +968,96 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     EpiStoreBF16::Params sp{reinterpret_cast<__nv_bfloat16*>(dx), d_in, 1.0f, 0};
     cudaError_t e = launch_gemm_pair<PairCfg<256, false, true>, EpiStoreBF16>(a, sp, p.sms, st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: dx");
+  }
+  return DORA_OK;
+}
+
+// Full (non-detached) gradient: the detached backward, then per row the
+// A.1 projection term, kappa_n = g_n dm_n / C_n:
+//   dB -= s diag(kappa) Q,       Q = W0 A^T + s B G  ([W0 | B | B] [A | sG_hi | sG_lo]^T)
+//   dA -= s [(kappa B)^T W0 + H A],   H = s B^T diag(kappa) B
+dora_status_t bf16_backward_full(const dora_desc_t& d, const Plan& p, int64_t T, const void* dy, const void* x,
+                                 const void* W0, const void* A, const void* B, const float* C, const float* g,
+                                 const void* su, const void* pre, float* dm, void* dA, void* dB, void* dx,
+                                 uint8_t* ws, cudaStream_t st) {
+  dora_status_t status = bf16_backward(d, p, T, dy, x, W0, A, B, C, g, su, pre, dm, dA, dB, dx, ws, st);
+  if (status != DORA_OK || T == 0) return status;  // no tokens: dm = 0, so kappa = 0
+  const int r = (int)d.r, d_in = (int)d.d_in, d_out = (int)d.d_out;
+  const int rp = (int)ceil_div(r, kBK) * kBK;
+  float* kappa = reinterpret_cast<float*>(ws + p.off_kappa);
+  __nv_bfloat16* Bk = reinterpret_cast<__nv_bfloat16*>(ws + p.off_bk);
+  __nv_bfloat16* gs = reinterpret_cast<__nv_bfloat16*>(ws + p.off_gs);
+  __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(ws + p.off_h);
+  float* qpart = reinterpret_cast<float*>(ws + p.off_q_part);
+  cudaError_t e;
+  {
+    const long long total = (long long)d_out * (r / 8);
+    ProfRange pr("full_kappa", st);
+    e = launch_pdl(full_kappa_kernel, dim3((unsigned)std::min<long long>(ceil_div(total, 256), 2048)), dim3(256), 0,
+                   st, g, (const float*)dm, C, reinterpret_cast<const __nv_bfloat16*>(B), d_out, r, kappa, Bk);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_status(e, "dora_backward_full: kappa");
+  }
+  // s G as bf16 hi + lo, then Q = W0 A^T + s B G into fp32 split partials.
+  e = gram_hi_lo(d, p, A, d.s, reinterpret_cast<float*>(ws + p.off_gram_part), gs, st);
+  if (e != cudaSuccess) return gemm_status(e, "dora_backward_full: Gram");
+  {
+    GemmArgs a;
+    a.a0 = Mat{W0, d_out, d_in, d_in};
+    a.a1 = Mat{B, d_out, r, r};
+    a.b0 = Mat{A, r, d_in, d_in};
+    a.b1 = Mat{gs, r, 2 * rp, 2 * rp};
+    a.K0 = d_in;
+    a.K1 = 2 * rp;
+    a.a1_kwrap = rp;
+    a.M = d_out;
+    a.N = r;
+    a.split = p.q;
+    a.name = "full_q_gemm";
+    EpiPartialTMA::Params pp;
+    if (!make_map_f32_3d(&pp.map, qpart, r, d_out, p.q.splits, 32, 32))
+      return gemm_status(cudaErrorInvalidValue, "dora_backward_full: Q");
+    e = pair_gemm_bn<false, false, EpiPartialTMA>(p.q_bn, a, pp, p.sms, st);
+    if (e != cudaSuccess) return gemm_status(e, "dora_backward_full: Q");
+    const long long total = (long long)d_out * (r / 4);
+    ProfRange pr("full_dB", st);
+    e = launch_pdl(full_dB_kernel, dim3((unsigned)std::min<long long>(ceil_div(total, 256), 148LL * 16)), dim3(256),
+                   0, st, (const float*)qpart, p.q.splits, (long long)d_out * r, d_out, r, (const float*)kappa, d.s,
+                   reinterpret_cast<__nv_bfloat16*>(dB));
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_status(e, "dora_backward_full: dB correction");
+  }
+  // H = s (kappa B)^T B  (both operands read MN-major from their [d_out x r] storage; K = d_out)
+  {
+    GemmArgs a;
+    a.a0 = Mat{Bk, d_out, r, r};
+    a.b0 = Mat{B, d_out, r, r};
+    a.K0 = d_out;
+    a.M = r;
+    a.N = r;
+    a.split = p.h;
+    a.name = "full_h_gemm";
+    e = narrow_gemm_1cta<true, true>(p.h_bn, a, d.s, H, r, false, reinterpret_cast<float*>(ws + p.off_h_part),
+                                     "full_h_reduce", st);
+    if (e != cudaSuccess) return gemm_status(e, "dora_backward_full: H");
+  }
+  // dA += -s [(kappa B)^T | H] [W0 ; A]  (M = r; A operands MN-major: kappa B as stored, H symmetric)
+  {
+    GemmArgs a;
+    a.a0 = Mat{Bk, d_out, r, r};
+    a.a1 = Mat{H, r, r, r};
+    a.b0 = Mat{W0, d_out, d_in, d_in};
+    a.b1 = Mat{A, r, d_in, d_in};
+    a.K0 = d_out;
+    a.K1 = r;
+    a.M = r;
+    a.N = d_in;
+    a.split.splits = 1;
+    a.split.kb_per_split = (int)(ceil_div(d_out, kBK) + ceil_div(r, kBK));
+    a.name = "full_dA_gemm";
+    EpiAxpyBF16::Params ap{reinterpret_cast<__nv_bfloat16*>(dA), d_in, -d.s};
+    e = launch_gemm_pair<PairCfg<256, true, true>, EpiAxpyBF16>(a, ap, p.sms, st);
+    if (e != cudaSuccess) return gemm_status(e, "dora_backward_full: dA correction");
   }
   return DORA_OK;
 }

@@ -242,3 +242,67 @@ dora_status_t f32_backward(const dora_desc_t& d, const Plan& p, int64_t T, const
 }
 
 }  // namespace dora
+
+namespace dora {
+
+// kappa_n = g_n dm_n / C_n and Bk[n][c] = kappa_n B[n][c].
+__global__ void f32_kappa_kernel(const float* __restrict__ g, const float* __restrict__ dm,
+                                 const float* __restrict__ C, const float* __restrict__ B, int d_out, int r,
+                                 float* __restrict__ kappa, float* __restrict__ Bk) {
+  const long long total = (long long)d_out * r;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int n = (int)(i / r), c = (int)(i % r);
+    const float k = g[n] * dm[n] / C[n];
+    if (c == 0) kappa[n] = k;
+    Bk[i] = k * B[i];
+  }
+}
+
+// dB[n][c] -= s kappa_n Q[n][c].
+__global__ void f32_full_dB_kernel(const float* __restrict__ Q, const float* __restrict__ kappa, int d_out, int r,
+                                   float s, float* __restrict__ dB) {
+  const long long total = (long long)d_out * r;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x)
+    dB[i] = fmaf(-s * kappa[i / r], Q[i], dB[i]);
+}
+
+// Full (non-detached) gradient, fp32: the detached backward, then
+//   dB -= s diag(kappa) (W0 A^T + s B G),  G = A A^T
+//   dA -= s (kappa B)^T W0 + s^2 (B^T diag(kappa) B) A
+dora_status_t f32_backward_full(const dora_desc_t& d, const Plan& p, int64_t T, const float* dy, const float* x,
+                                const float* W0, const float* A, const float* B, const float* C, const float* g,
+                                const float* su, const float* pre, float* dm, float* dA, float* dB, float* dx,
+                                uint8_t* ws, cudaStream_t st) {
+  dora_status_t status = f32_backward(d, p, T, dy, x, W0, A, B, C, g, su, pre, dm, dA, dB, dx, ws, st);
+  if (status != DORA_OK || T == 0) return status;  // no tokens: dm = 0, so kappa = 0
+  const int r = (int)d.r, d_in = (int)d.d_in, d_out = (int)d.d_out;
+  float* kappa = reinterpret_cast<float*>(ws + p.off_kappa);
+  float* Bk = reinterpret_cast<float*>(ws + p.off_bk);
+  float* G = reinterpret_cast<float*>(ws + p.off_gs);
+  float* Q = reinterpret_cast<float*>(ws + p.off_q_part);
+  float* H = reinterpret_cast<float*>(ws + p.off_h);
+  const long long n = (long long)d_out * r;
+  {
+    ProfRange pr("f32_full_kappa", st);
+    f32_kappa_kernel<<<(unsigned)std::min<long long>(cdiv(n, 256), 4096), 256, 0, st>>>(g, dm, C, B, d_out, r, kappa,
+                                                                                         Bk);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = sgemm(r, r, d_in, A, d_in, 1, A, d_in, 1, G, r, 1.f, 0.f, st);            // G = A A^T
+  if (e == cudaSuccess) e = sgemm(d_out, r, d_in, W0, d_in, 1, A, d_in, 1, Q, r, 1.f, 0.f, st);       // Q = W0 A^T
+  if (e == cudaSuccess) e = sgemm(d_out, r, r, B, r, 1, G, r, 1, Q, r, d.s, 1.f, st);                 //   + s B G
+  if (e == cudaSuccess) {
+    ProfRange pr("f32_full_dB", st);
+    f32_full_dB_kernel<<<(unsigned)std::min<long long>(cdiv(n, 256), 4096), 256, 0, st>>>(Q, kappa, d_out, r, d.s,
+                                                                                           dB);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) e = sgemm(r, r, d_out, Bk, 1, r, B, 1, r, H, r, 1.f, 0.f, st);                 // H = (kB)^T B
+  if (e == cudaSuccess) e = sgemm(r, d_in, d_out, Bk, 1, r, W0, 1, d_in, dA, d_in, -d.s, 1.f, st);     // dA -= s (kB)^T W0
+  if (e == cudaSuccess) e = sgemm(r, d_in, r, H, r, 1, A, 1, d_in, dA, d_in, -d.s * d.s, 1.f, st);     //    - s^2 H A
+  return cuda_status(e, "dora_backward_full (fp32)");
+}
+
+}  // namespace dora

@@ -34,6 +34,10 @@ struct Plan {
   Split du, dB, dA;
   int du_bn = 0, dB_bn = 0, dA_bn = 0;
   size_t off_dz = 0, off_dm_part = 0, off_du_part = 0, off_du = 0, off_dB_part = 0, off_dA_part = 0;
+  // full (non-detached) gradient: kappa, kappa-scaled B, Gram, Q = W' A^T, H = s B^T diag(kappa) B
+  Split q, h;
+  int q_bn = 0, h_bn = 0;
+  size_t off_kappa = 0, off_bk = 0, off_q_part = 0, off_h_part = 0, off_h = 0;
   // split counters (+ padding that must start at zero), cleared by one memset per call
   size_t off_ctr = 0, zero_bytes = 0;
   int gram_tiles = 0;
@@ -72,6 +76,11 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
                             const void* su, const void* pre, float* dm, void* dA, void* dB, void* dx,
                             uint8_t* ws, cudaStream_t st);
 
+dora_status_t bf16_backward_full(const dora_desc_t& d, const Plan& p, int64_t T, const void* dy, const void* x,
+                                 const void* W0, const void* A, const void* B, const float* C, const float* g,
+                                 const void* su, const void* pre, float* dm, void* dA, void* dB, void* dx,
+                                 uint8_t* ws, cudaStream_t st);
+
 dora_status_t bf16_merge(const dora_desc_t& d, const Plan& p, const void* W0, const void* A, const void* B,
                          const float* g, void* W_out, uint8_t* ws, cudaStream_t st);
 
@@ -85,6 +94,11 @@ dora_status_t f32_backward(const dora_desc_t& d, const Plan& p, int64_t T, const
                            const float* W0, const float* A, const float* B, const float* C, const float* g,
                            const float* su, const float* pre, float* dm, float* dA, float* dB, float* dx,
                            uint8_t* ws, cudaStream_t st);
+
+dora_status_t f32_backward_full(const dora_desc_t& d, const Plan& p, int64_t T, const float* dy, const float* x,
+                                const float* W0, const float* A, const float* B, const float* C, const float* g,
+                                const float* su, const float* pre, float* dm, float* dA, float* dB, float* dx,
+                                uint8_t* ws, cudaStream_t st);
 
 // Brackets one kernel launch with profiling events when profiling is on.
 class ProfRange {

@@ -60,7 +60,13 @@ typedef enum {
 
 typedef enum { DORA_BF16 = 0, DORA_FP32 = 1 } dora_dtype_t;
 
-typedef enum { DORA_OP_NORM = 0, DORA_OP_FORWARD = 1, DORA_OP_BACKWARD = 2, DORA_OP_MERGE = 3 } dora_op_t;
+typedef enum {
+  DORA_OP_NORM = 0,
+  DORA_OP_FORWARD = 1,
+  DORA_OP_BACKWARD = 2,
+  DORA_OP_MERGE = 3,
+  DORA_OP_BACKWARD_FULL = 4
+} dora_op_t;
 
 typedef struct {
   int64_t d_out;      /* output features (rows of W0, B, entries of m)   */
@@ -149,6 +155,26 @@ DORA_API dora_status_t dora_backward(const dora_desc_t* desc, int64_t T, const v
                             const void* A, const void* B, const float* norm, const float* g, const void* su_save,
                             const void* pre_save, float* dm, void* dA, void* dB, void* dx, void* ws,
                             size_t ws_bytes, dora_stream_t stream);
+
+/*
+ * dora_backward_full -- the same gradients without the detach of the norm.
+ *
+ * DoRA notes appendix A eq. (A.1): through C the gradient of V'_n is
+ * (m_n / C_n) (I - V'_n V'_n^T / C_n^2) grad W'_n. With
+ * kappa_n = g_n dm_n / C_n (= m_n dm_n / C_n^2, dm as above) this is the
+ * detached gradient minus kappa_n V'_n per row, V' = W0 + s B A, so
+ *   dB_full = dB - s diag(kappa) (W0 A^T + s B A A^T)
+ *   dA_full = dA - s (diag(kappa) B)^T W0 - s^2 (B^T diag(kappa) B) A
+ * while dm and dx are unchanged (they do not pass through C). The dense V' is
+ * never formed: the two extra products re-read W0 once each.
+ * Arguments, layouts and errors as dora_backward; workspace from
+ * dora_workspace_size(desc, T, DORA_OP_BACKWARD_FULL).
+ */
+DORA_API dora_status_t dora_backward_full(const dora_desc_t* desc, int64_t T, const void* dy, const void* x,
+                                          const void* W0, const void* A, const void* B, const float* norm,
+                                          const float* g, const void* su_save, const void* pre_save, float* dm,
+                                          void* dA, void* dB, void* dx, void* ws, size_t ws_bytes,
+                                          dora_stream_t stream);
 
 /*
  * dora_merge -- the merged deployment weight W' = diag(g) (W0 + s B A).

@@ -138,3 +138,23 @@ def test_merge_validation(lib):
     bad = _desc(r=12)
     st = lib.dora_merge(ctypes.byref(bad), fake, fake, fake, fake, fake, None, 0, None)
     assert st == 1
+
+
+@pytest.mark.parametrize("key", sorted(WORKLOADS))
+def test_full_backward_workspace(lib, key):
+    wl = WORKLOADS[key]
+    dt = 0 if wl.dtype == "bf16" else 1
+    d = _desc(wl.d_out, wl.d_in, wl.r, dt, wl.s)
+    det = lib.dora_workspace_size(ctypes.byref(d), wl.T, 2)
+    full = lib.dora_workspace_size(ctypes.byref(d), wl.T, 4)
+    # The full gradient adds kappa, kappa * B and the Q = W' A^T partials (at least d_out x r fp32).
+    assert full >= det + wl.d_out * wl.r * 4
+    assert lib.dora_workspace_size(ctypes.byref(d), 0, 4) == 0
+
+
+def test_full_backward_validation(lib):
+    d = _desc()
+    fake = ctypes.c_void_p(4096)
+    st = lib.dora_backward_full(ctypes.byref(d), 8, fake, fake, fake, fake, fake, fake, fake, None, fake, fake, fake,
+                                fake, fake, fake, 1 << 30, None)
+    assert st == 1 and "su_save" in dw.dora_last_error()
