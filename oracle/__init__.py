@@ -13,6 +13,8 @@ Sources (cited by page and equation):
                   steps 7-14 and 16-17; gradients eq. (7) and eq. (8); the
                   detach trick of section 3.4; the full gradient eq. (A.1)
                   and the dropped term (A.2) of appendix A.
+                  Section 3.5: DVoRA, the direction update taken from VeRA,
+                  diag(b) B_shared diag(d) A_shared with the shared pair frozen.
   [Scaling DoRA]  "Scaling DoRA" (gptget.net/papers/2603.22276), English
                   abstract: the row-wise norm of W + sBA with W of shape
                   [d_out, d_in], and the g - 1 near-unity rescaling regime.
@@ -37,7 +39,7 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["adapted_direction", "norm", "forward", "backward", "merge"]
+__all__ = ["adapted_direction", "norm", "forward", "backward", "merge", "vera_direction", "vera_gradients"]
 
 
 def _f64(a) -> np.ndarray:
@@ -120,3 +122,25 @@ def merge(W0, A, B, m, s: float) -> np.ndarray:
     """
     V = adapted_direction(W0, A, B, s)
     return (_f64(m) / _row_norms(V))[:, None] * V
+
+
+def vera_direction(B_shared, b, d) -> np.ndarray:
+    """B' = diag(b) @ B_shared @ diag(d), [d_out x r].
+
+    [DoRA notes] section 3.5 (DVoRA): the per-layer update is
+    diag(b) B_shared diag(d) A_shared, so DVoRA is DoRA with B = B' and
+    A = A_shared; norm, forward, backward and merge apply unchanged.
+    """
+    return _f64(b)[:, None] * _f64(B_shared) * _f64(d)[None, :]
+
+
+def vera_gradients(dBp, B_shared, b, d):
+    """Gradients of the two trained vectors from dB' = dL/dB' (chain rule through B').
+
+    [DoRA notes] section 3.5: only b, d (and the magnitude m) are trained;
+    A_shared and B_shared are frozen. With B'[n, c] = b[n] B_shared[n, c] d[c]:
+      db[n] = sum_c dB'[n, c] B_shared[n, c] d[c]
+      dd[c] = sum_n dB'[n, c] b[n] B_shared[n, c]
+    """
+    P = _f64(dBp) * _f64(B_shared)
+    return P @ _f64(d), _f64(b) @ P

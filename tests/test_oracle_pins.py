@@ -23,6 +23,11 @@ What pins what:
   a2_term     detached minus full dV equals the dropped term (A.2)
   eq8         dm_n = |grad W'_n| cos(grad W'_n, V'_n) (eq. (8), second form)
   near_unity  m = C (1 + delta) gives g - 1 = delta
+  vera_fd     DVoRA (DoRA notes sec. 3.5): finite differences of L in the
+              trained vectors b and d, with the norm held fixed and free, give
+              vera_gradients of the detached and the full dB'
+  vera_unit   b = 1 and d = 1 reduce DVoRA to DoRA with B = B_shared, and
+              B' scales each row by b and each column by d
 """
 import json
 import os
@@ -216,8 +221,34 @@ def pin_near_unity(orc):
     _close(g, 1.0 + delta, 1e-15, "g = 1 + delta")
 
 
+def pin_vera_fd(orc):
+    rng = np.random.default_rng(21)
+    L = _rand_layer(rng, 4, 5, 3, 3)
+    Bs = L["B"]
+    b, d = rng.uniform(0.5, 1.5, 4), rng.uniform(-1.0, 1.0, 3)
+    W0, A, m, s, x, dy = (L[k] for k in ("W0", "A", "m", "s", "x", "dy"))
+    C0, _, _ = orc.norm(W0, A, orc.vera_direction(Bs, b, d), m, s)
+    for full in (False, True):
+        Cf = None if full else C0
+        loss = lambda: float(np.sum(dy * orc.forward(x, W0, A, orc.vera_direction(Bs, b, d), m, s, C=Cf)))
+        dBp = orc.backward(dy, x, W0, A, orc.vera_direction(Bs, b, d), m, s, full=full)["dB"]
+        db, dd = orc.vera_gradients(dBp, Bs, b, d)
+        _close(db, _fd(loss, b), 1e-7, f"db vs FD (full={full})")
+        _close(dd, _fd(loss, d), 1e-7, f"dd vs FD (full={full})")
+
+
+def pin_vera_unit(orc):
+    rng = np.random.default_rng(22)
+    Bs = rng.standard_normal((5, 3))
+    _close(orc.vera_direction(Bs, np.ones(5), np.ones(3)), Bs, 0.0, "b = d = 1 gives B_shared")
+    b, d = rng.uniform(0.5, 2.0, 5), rng.uniform(0.5, 2.0, 3)
+    Bp = orc.vera_direction(Bs, b, d)
+    _close(Bp[2] / Bs[2], b[2] * d, 1e-15, "row 2 scaled by b_2 d")
+    _close(Bp[:, 1] / Bs[:, 1], b * d[1], 1e-15, "column 1 scaled by b d_1")
+
+
 PINS = [pin_golden, pin_factored, pin_zero_B, pin_init, pin_scale, pin_merge, pin_fd_x_m,
-        pin_fd_detached, pin_fd_full, pin_a2_term, pin_eq8, pin_near_unity]
+        pin_fd_detached, pin_fd_full, pin_a2_term, pin_eq8, pin_near_unity, pin_vera_fd, pin_vera_unit]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -270,7 +301,8 @@ def test_near_unity_generator():
 
 def _mutant(**overrides):
     ns = types.SimpleNamespace(adapted_direction=oracle.adapted_direction, norm=oracle.norm,
-                               forward=oracle.forward, backward=oracle.backward, merge=oracle.merge)
+                               forward=oracle.forward, backward=oracle.backward, merge=oracle.merge,
+                               vera_direction=oracle.vera_direction, vera_gradients=oracle.vera_gradients)
     for k, v in overrides.items():
         setattr(ns, k, v)
     return ns
@@ -346,6 +378,10 @@ MUTANTS = {
     "dA_without_s": _mutant(backward=_backward_variant("dA_no_s")),
     "dx_without_g": _mutant(backward=_backward_variant("dx_no_g")),
     "dx_from_W0_only": _mutant(backward=_backward_variant("dx_W0_only")),
+    "vera_b_d_swapped": _mutant(vera_direction=lambda Bs, b, d: np.asarray(Bs, float) * np.outer(
+        np.resize(np.asarray(d, float), len(b)), np.resize(np.asarray(b, float), len(d)))),
+    "vera_dd_missing_b": _mutant(vera_gradients=lambda dBp, Bs, b, d: (
+        (np.asarray(dBp) * Bs) @ np.asarray(d, float), np.sum(np.asarray(dBp) * Bs, axis=0))),
 }
 
 
