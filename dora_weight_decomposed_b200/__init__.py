@@ -11,6 +11,8 @@ every call raises.
     y, su, pre   = dora_forward(x, W0, A, B, gm1, s)
     dm, dA, dB, dx = dora_backward(dy, x, W0, A, B, norm, g, su, pre, s)    # full=True: no detach
     W_merged     = dora_merge(W0, A, B, g, s)
+    B_vera       = dora_vera_compose(B_shared, b, d)       # DVoRA: B' for the calls above
+    db, dd       = dora_vera_grad(B_shared, b, d, dB)
 
 bf16 tensors use the tcgen05 tensor-core path; fp32 tensors use the SIMT path.
 """
@@ -21,7 +23,8 @@ import os
 import threading
 
 __all__ = ["DoraError", "load_library", "library_path", "dora_workspace_size", "dora_norm", "dora_forward",
-           "dora_norm_noalloc", "dora_backward", "dora_backward_full", "dora_merge", "dora_device_status", "dora_last_error",
+           "dora_norm_noalloc", "dora_backward", "dora_backward_full", "dora_merge", "dora_vera_compose",
+           "dora_vera_grad", "dora_device_status", "dora_last_error",
            "dora_version",
            "dora_profile_start",
            "dora_profile_stop", "dora_profile_count", "dora_profile_read", "DORA_OP_NORM",
@@ -29,11 +32,11 @@ __all__ = ["DoraError", "load_library", "library_path", "dora_workspace_size", "
            "EXPORTED_SYMBOLS"]
 
 DORA_BF16, DORA_FP32 = 0, 1
-DORA_OP_NORM, DORA_OP_FORWARD, DORA_OP_BACKWARD, DORA_OP_MERGE, DORA_OP_BACKWARD_FULL = 0, 1, 2, 3, 4
+DORA_OP_NORM, DORA_OP_FORWARD, DORA_OP_BACKWARD, DORA_OP_MERGE, DORA_OP_BACKWARD_FULL, DORA_OP_VERA_GRAD = range(6)
 STATUS_NAMES = {0: "DORA_OK", 1: "DORA_EINVAL", 2: "DORA_EUNSUPPORTED", 3: "DORA_EWORKSPACE", 4: "DORA_ECUDA",
                 5: "DORA_ETIMEOUT"}
 EXPORTED_SYMBOLS = ("dora_workspace_size", "dora_norm", "dora_norm_noalloc", "dora_forward", "dora_backward",
-                    "dora_backward_full", "dora_merge", "dora_device_status",
+                    "dora_backward_full", "dora_merge", "dora_vera_compose", "dora_vera_grad", "dora_device_status",
                     "dora_profile_start", "dora_profile_stop", "dora_profile_count", "dora_profile_read",
                     "dora_last_error", "dora_version")
 
@@ -87,6 +90,10 @@ def load_library() -> ctypes.CDLL:
         lib.dora_backward_full.restype = ctypes.c_int
         lib.dora_merge.argtypes = [DP, P, P, P, P, P, P, SZ, P]
         lib.dora_merge.restype = ctypes.c_int
+        lib.dora_vera_compose.argtypes = [DP, P, P, P, P, P]
+        lib.dora_vera_compose.restype = ctypes.c_int
+        lib.dora_vera_grad.argtypes = [DP, P, P, P, P, P, P, P, SZ, P]
+        lib.dora_vera_grad.restype = ctypes.c_int
         lib.dora_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint)]
         lib.dora_device_status.restype = ctypes.c_int
         lib.dora_profile_start.argtypes = [ctypes.c_int]
@@ -332,3 +339,36 @@ def dora_norm_noalloc(W0, A, B, m, s: float, *, norm_out=None, g_out=None, gm1_o
 def dora_backward_full(dy, x, W0, A, B, norm, g, su_save, pre_save, s: float, **kw):
     """dora_backward with the gradient through the norm kept (appendix A eq. A.1)."""
     return dora_backward(dy, x, W0, A, B, norm, g, su_save, pre_save, s, full=True, **kw)
+
+
+def dora_vera_compose(B_shared, b, d, *, out=None, s: float = 1.0, stream=None):
+    """DVoRA's B' = diag(b) B_shared diag(d) [d_out x r]; b, d float32."""
+    torch = _torch()
+    lib = load_library()
+    d_out, r = B_shared.shape
+    _shape(b, (d_out,), "b")
+    _shape(d, (r,), "d")
+    if b.dtype != torch.float32 or d.dtype != torch.float32:
+        raise TypeError("b and d are float32")
+    desc = _desc(d_out, 8, r, B_shared.dtype, s)
+    out = torch.empty_like(B_shared) if out is None else out
+    _check(lib.dora_vera_compose(ctypes.byref(desc), _ptr(B_shared), _ptr(b), _ptr(d), _ptr(out),
+                                 _stream_ptr(stream)))
+    return out
+
+
+def dora_vera_grad(B_shared, b, d, dB, *, s: float = 1.0, ws=None, stream=None):
+    """Gradients (db [d_out], dd [r], float32) of DVoRA's trained vectors from dB' = dL/dB'."""
+    torch = _torch()
+    lib = load_library()
+    d_out, r = B_shared.shape
+    _shape(b, (d_out,), "b")
+    _shape(d, (r,), "d")
+    _shape(dB, (d_out, r), "dB")
+    desc = _desc(d_out, 8, r, B_shared.dtype, s)
+    db = torch.empty(d_out, dtype=torch.float32, device=B_shared.device)
+    dd = torch.empty(r, dtype=torch.float32, device=B_shared.device)
+    wsb, nbytes = _workspace(desc, 0, DORA_OP_VERA_GRAD, B_shared.device, ws)
+    _check(lib.dora_vera_grad(ctypes.byref(desc), _ptr(B_shared), _ptr(b), _ptr(d), _ptr(dB), _ptr(db), _ptr(dd),
+                              _ptr(wsb), nbytes, _stream_ptr(stream)))
+    return db, dd

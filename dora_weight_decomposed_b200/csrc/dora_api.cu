@@ -235,6 +235,10 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
       }
     }
   }
+  if (op == DORA_OP_VERA_GRAD) {
+    p.vera_blocks = (int)std::min<int64_t>(cdiv(d_out, 64), 296);
+    p.off_f32_a = take((size_t)p.vera_blocks * r * 4);
+  }
   p.total = off;
   return p;
 }
@@ -317,8 +321,35 @@ using namespace dora;
 extern "C" {
 
 size_t dora_workspace_size(const dora_desc_t* desc, int64_t T, int op) {
-  if (!check_desc(desc) || !check_T(T) || op < DORA_OP_NORM || op > DORA_OP_BACKWARD_FULL) return 0;
+  if (!check_desc(desc) || !check_T(T) || op < DORA_OP_NORM || op > DORA_OP_VERA_GRAD) return 0;
   return make_plan(*desc, T, op).total;
+}
+
+dora_status_t dora_vera_compose(const dora_desc_t* desc, const void* B_shared, const float* b, const float* d,
+                                void* B_out, dora_stream_t stream) {
+  if (!check_desc(desc)) return DORA_EINVAL;
+  const size_t al = tensor_align(desc);
+  if (!check_ptr(B_shared, "B_shared", al) || !check_ptr(b, "b", 4) || !check_ptr(d, "d", 4) ||
+      !check_ptr(B_out, "B_out", al))
+    return DORA_EINVAL;
+  dora_status_t s = check_device(desc);
+  if (s != DORA_OK) return s;
+  return vera_compose(*desc, B_shared, b, d, B_out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dora_status_t dora_vera_grad(const dora_desc_t* desc, const void* B_shared, const float* b, const float* d,
+                             const void* dB, float* db, float* dd, void* ws, size_t ws_bytes, dora_stream_t stream) {
+  if (!check_desc(desc)) return DORA_EINVAL;
+  const size_t al = tensor_align(desc);
+  if (!check_ptr(B_shared, "B_shared", al) || !check_ptr(b, "b", 4) || !check_ptr(d, "d", 4) ||
+      !check_ptr(dB, "dB", al) || !check_ptr(db, "db", 4) || !check_ptr(dd, "dd", 4))
+    return DORA_EINVAL;
+  const Plan p = make_plan(*desc, 0, DORA_OP_VERA_GRAD);
+  dora_status_t s = check_ws(p, ws, ws_bytes);
+  if (s != DORA_OK) return s;
+  if ((s = check_device(desc)) != DORA_OK) return s;
+  return vera_grad(*desc, p, B_shared, b, d, dB, db, dd, reinterpret_cast<uint8_t*>(ws),
+                   reinterpret_cast<cudaStream_t>(stream));
 }
 
 dora_status_t dora_merge(const dora_desc_t* desc, const void* W0, const void* A, const void* B, const float* g,

@@ -38,6 +38,8 @@ struct Plan {
   Split q, h;
   int q_bn = 0, h_bn = 0;
   size_t off_kappa = 0, off_bk = 0, off_q_part = 0, off_h_part = 0, off_h = 0;
+  // DVoRA gradient: row blocks of the dd partial sums (scratch in off_f32_a)
+  int vera_blocks = 0;
   // split counters (+ padding that must start at zero), cleared by one memset per call
   size_t off_ctr = 0, zero_bytes = 0;
   int gram_tiles = 0;
@@ -99,6 +101,12 @@ dora_status_t f32_backward_full(const dora_desc_t& d, const Plan& p, int64_t T, 
                                 const float* W0, const float* A, const float* B, const float* C, const float* g,
                                 const float* su, const float* pre, float* dm, float* dA, float* dB, float* dx,
                                 uint8_t* ws, cudaStream_t st);
+
+// DVoRA (both dtypes): B' = diag(b) B_shared diag(d), and db, dd from dB'.
+dora_status_t vera_compose(const dora_desc_t& d, const void* Bs, const float* b, const float* dv, void* Bp,
+                           cudaStream_t st);
+dora_status_t vera_grad(const dora_desc_t& d, const Plan& p, const void* Bs, const float* b, const float* dv,
+                        const void* dBp, float* db, float* dd, uint8_t* ws, cudaStream_t st);
 
 // Brackets one kernel launch with profiling events when profiling is on.
 class ProfRange {

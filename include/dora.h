@@ -65,7 +65,8 @@ typedef enum {
   DORA_OP_FORWARD = 1,
   DORA_OP_BACKWARD = 2,
   DORA_OP_MERGE = 3,
-  DORA_OP_BACKWARD_FULL = 4
+  DORA_OP_BACKWARD_FULL = 4,
+  DORA_OP_VERA_GRAD = 5
 } dora_op_t;
 
 typedef struct {
@@ -175,6 +176,31 @@ DORA_API dora_status_t dora_backward_full(const dora_desc_t* desc, int64_t T, co
                                           const float* g, const void* su_save, const void* pre_save, float* dm,
                                           void* dA, void* dB, void* dx, void* ws, size_t ws_bytes,
                                           dora_stream_t stream);
+
+/*
+ * DVoRA -- DoRA notes section 3.5: the direction update of VeRA,
+ * diag(b) B_shared diag(d) A_shared, with the random pair A_shared [r x d_in],
+ * B_shared [d_out x r] shared and frozen, and only b [d_out], d [r] (and m)
+ * trained. The layer is DoRA with A = A_shared and B = B' = diag(b) B_shared
+ * diag(d): form B' with dora_vera_compose, run dora_norm / dora_forward /
+ * dora_backward (or _full) / dora_merge on it unchanged, and turn the dB' they
+ * return into the gradients of b and d with dora_vera_grad (dA is then not
+ * needed: A_shared is frozen).
+ *
+ * dora_vera_compose: B_out[n][c] = b[n] B_shared[n][c] d[c], computed in fp32
+ *   and rounded once to the desc dtype. B_shared, B_out [d_out x r] (dtype);
+ *   b [d_out], d [r] fp32. No workspace.
+ * dora_vera_grad: db[n] = sum_c dB[n][c] B_shared[n][c] d[c] and
+ *   dd[c] = sum_n dB[n][c] b[n] B_shared[n][c], fp32, deterministic. dB is the
+ *   gradient of B' [d_out x r] (dtype); db [d_out], dd [r] fp32 out.
+ *   Workspace: dora_workspace_size(desc, 0, DORA_OP_VERA_GRAD).
+ * Both read d_out, r and dtype from desc; desc->d_in and desc->s are not used.
+ */
+DORA_API dora_status_t dora_vera_compose(const dora_desc_t* desc, const void* B_shared, const float* b, const float* d,
+                                         void* B_out, dora_stream_t stream);
+DORA_API dora_status_t dora_vera_grad(const dora_desc_t* desc, const void* B_shared, const float* b, const float* d,
+                                      const void* dB, float* db, float* dd, void* ws, size_t ws_bytes,
+                                      dora_stream_t stream);
 
 /*
  * dora_merge -- the merged deployment weight W' = diag(g) (W0 + s B A).
