@@ -97,7 +97,7 @@ def kernel_work(name, wl):
 # valid only while these files are unchanged.
 KERNEL_SOURCES = {
     "fwd_compose_gemm": ("sm100_ptx.cuh", "gemm_sm100.cuh", "dora_bf16.cu"),
-    "merge_gemm": ("sm100_ptx.cuh", "gemm_sm100.cuh", "merge_sm100.cuh", "dora_bf16.cu"),
+    "merge_gemm": ("sm100_ptx.cuh", "gemm_sm100.cuh", "merge_sm100.cuh"),
 }
 
 

@@ -871,8 +871,7 @@ dora_status_t bf16_merge(const dora_desc_t& d, const Plan& p, const void* W0, co
   const MergeGeom geom{(int)d.d_out, (int)d.d_in, kb, g, d.s, reinterpret_cast<const __nv_bfloat16*>(W0),
                        reinterpret_cast<__nv_bfloat16*>(W_out)};
   const long long items = ceil_div(d.d_out, 2 * kBM) * ceil_div(d.d_in, 256);
-  const long long pairs = std::max<long long>(1, std::min<long long>(items, p.sms / 2));
-  cudaError_t e = launch_merge<MergeCfg<4, 6>>(ta, tb, geom, pairs, st);
+  cudaError_t e = launch_merge<MergeLaunchCfg>(ta, tb, geom, merge_pairs(items, p.sms), st);
   if (e == cudaSuccess) e = cudaGetLastError();
   return gemm_status(e, "dora_merge");
 }

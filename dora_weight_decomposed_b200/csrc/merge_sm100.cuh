@@ -63,6 +63,14 @@ struct MergeCfg {
   static constexpr uint32_t TMEM_COLS = 512;
 };
 
+// The configuration dora_merge launches: 4 operand stages (128 KB), a ring of
+// 6 W0 pieces per epilogue warp (96 KB); one CTA pair per two SMs, at most
+// one per tile.
+using MergeLaunchCfg = MergeCfg<4, 6>;
+inline long long merge_pairs(long long tiles, int sms) {
+  return tiles < sms / 2 ? (tiles > 0 ? tiles : 1) : (sms / 2 > 0 ? sms / 2 : 1);
+}
+
 struct MergeGeom {
   int M, N, kb;  // d_out, d_in, k-blocks of r
   const float* g;
