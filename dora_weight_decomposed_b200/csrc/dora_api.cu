@@ -151,7 +151,6 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
   if (d.dtype == DORA_BF16) {
     const double kbB = 64.0 * 2.0;  // bytes per K element pair of rows (x 64 K per k-block)
     if (op == DORA_OP_NORM) {
-      const int bk = bn_narrow_k(r);
       // The Gram GEMM (CTA pairs, one tile column) is small: split K over the
       // pairs, with its fp32 partials capped at 8 MiB.
       p.gram_bn = bn_pair_k(r);
@@ -159,13 +158,15 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
       p.gram = choose_split(cdiv(r, 256), cdiv(d_in, 64), p.sms / 2, kbB * (128 + p.gram_bn / 2.0), 0.0,
                             (double)r * r, gram_max);
       p.off_gram_part = take((size_t)p.gram.splits * r * r * 4);
-      p.norm = choose_split(cdiv(d_out, 128), cdiv(d_in, 64) + 2 * cdiv(r, 64), p.sms, kbB * (128 + bk), 0.0,
-                            (double)d_out);
+      // The norm GEMM runs on CTA pairs, 256 rows x the whole rank per tile.
+      p.norm_bn = bn_pair_k(r);
+      p.norm = choose_split(cdiv(d_out, 256), cdiv(d_in, 64) + 2 * cdiv(r, 64), p.sms / 2,
+                            kbB * (128 + p.norm_bn / 2.0), 0.0, (double)d_out);
       p.off_norm_part = take((size_t)p.norm.splits * d_out * 4);
       p.off_gs = take((size_t)r * 2 * cdiv(r, 64) * 64 * 2);
-      // split counters of the norm's row tiles, zeroed by one memset per call
+      // split counters, one per 128-row half of a pair tile, zeroed by one memset per call
       p.gram_tiles = 0;
-      p.zero_bytes = (size_t)cdiv(d_out, 128) * 4;
+      p.zero_bytes = (size_t)2 * cdiv(d_out, 256) * 4;
       p.off_ctr = take(p.zero_bytes);
     } else if (op == DORA_OP_FORWARD && T > 0) {
       const NarrowChoice u = choose_narrow(T, r, d_in, false, p.sms);

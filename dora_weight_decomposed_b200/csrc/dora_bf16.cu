@@ -458,22 +458,58 @@ struct EpiAxpyBF16 {
   }
 };
 
-template <int BN>
-static cudaError_t norm_gemm_bn(const GemmArgs& g, const EpiNorm::Params& ep, cudaStream_t st) {
-  return launch_gemm<GemmCfg<BN, false, false>, EpiNorm>(g, ep, st);
+// Non-persistent CTA-pair launch: one 256 x BN tile and one K split per pair
+// (grid 2 x tiles, 1, splits).
+template <class Cfg, class Epi>
+static cudaError_t launch_gemm_pair_split(const GemmArgs& g, const typename Epi::Params& ep, cudaStream_t st) {
+  CUtensorMap ta0, ta1, tb0, tb1;
+  const int a_box = Cfg::A_MN ? 64 : kBM;
+  const int b_box = Cfg::B_MN ? 64 : Cfg::B_BOX;
+  t_detail.clear();
+  if (!make_map(&ta0, g.a0, a_box, "A source 0") || !make_map(&tb0, g.b0, b_box, "B source 0"))
+    return cudaErrorInvalidValue;
+  const int kb0 = (int)ceil_div(g.K0, kBK);
+  const int kb1 = g.K1 > 0 ? (int)ceil_div(g.K1, kBK) : 0;
+  if (kb1 > 0) {
+    if (!make_map(&ta1, g.a1, a_box, "A source 1") || !make_map(&tb1, g.b1, b_box, "B source 1"))
+      return cudaErrorInvalidValue;
+  } else {
+    ta1 = ta0;
+    tb1 = tb0;
+  }
+  const int kps = g.split.kb_per_split > 0 ? g.split.kb_per_split : kb0 + kb1;
+  GemmGeom geom{g.M, g.N, kb0, kb1, kps, g.a1_kwrap};
+  const long long splits = ceil_div(std::max(kb0 + kb1, 1), kps);
+  const long long tiles = ceil_div(g.N, Cfg::BN) * ceil_div(g.M, 2 * kBM);
+  auto kern = gemm_sm100_pair_split_kernel<Cfg, Epi>;
+  constexpr int smem_bytes = PairSplitLayout<Cfg, Epi>::SMEM_BYTES;
+  static std::atomic<unsigned long long> smem_set{0};
+  cudaError_t e = set_smem_once(smem_set, kern, smem_bytes);
+  if (e != cudaSuccess) {
+    t_detail = "shared-memory attribute (" + std::to_string(smem_bytes) + " bytes)";
+    return e;
+  }
+  {
+    ProfRange pr(g.name, st);
+    e = launch_pdl(kern, dim3((unsigned)(2 * tiles), 1, (unsigned)splits), dim3(kGemmThreads), smem_bytes, st, ta0,
+                   ta1, tb0, tb1, geom, ep);
+  }
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) t_detail = "pair split launch, " + std::to_string(tiles) + " tiles x " +
+                                   std::to_string(splits) + " splits";
+  return e;
 }
 
-
+// The factored norm GEMM on CTA pairs: 256 rows x the whole rank per tile.
 static cudaError_t norm_gemm(int bn, const GemmArgs& g, const EpiNorm::Params& ep, cudaStream_t st) {
   switch (bn) {
-    case 16: return norm_gemm_bn<16>(g, ep, st);
-    case 32: return norm_gemm_bn<32>(g, ep, st);
-    case 64: return norm_gemm_bn<64>(g, ep, st);
-    case 128: return norm_gemm_bn<128>(g, ep, st);
-    case 256: return norm_gemm_bn<256>(g, ep, st);
-    case 384: return norm_gemm_bn<384>(g, ep, st);
-    case 512: return norm_gemm_bn<512>(g, ep, st);
+    case 64: return launch_gemm_pair_split<PairCfg<64, false, false>, EpiNorm>(g, ep, st);
+    case 128: return launch_gemm_pair_split<PairCfg<128, false, false>, EpiNorm>(g, ep, st);
+    case 256: return launch_gemm_pair_split<PairCfg<256, false, false>, EpiNorm>(g, ep, st);
+    case 384: return launch_gemm_pair_split<PairCfg<384, false, false>, EpiNorm>(g, ep, st);
+    case 512: return launch_gemm_pair_split<PairCfg<512, false, false>, EpiNorm>(g, ep, st);
   }
+  t_detail = "no norm tile of width " + std::to_string(bn);
   return cudaErrorInvalidValue;
 }
 
@@ -804,7 +840,7 @@ dora_status_t bf16_norm(const dora_desc_t& d, const Plan& p, const void* W0, con
   na.name = "norm_gemm";
   EpiNorm::Params np{reinterpret_cast<const __nv_bfloat16*>(B), r, 2.0f * d.s, norm_part, d_out,
                      ctr + p.gram_tiles, m, C, g, gm1};
-  e = norm_gemm(bn_narrow_k(r), na, np, st);
+  e = norm_gemm(p.norm_bn, na, np, st);
   return gemm_status(e, "dora_norm: factored norm GEMM");
 }
 

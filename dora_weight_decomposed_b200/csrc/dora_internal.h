@@ -23,7 +23,7 @@ struct Plan {
   int sms = 148;
   // norm
   Split gram, norm;
-  int gram_bn = 0;
+  int gram_bn = 0, norm_bn = 0;
   size_t off_gram_part = 0, off_gs = 0, off_norm_part = 0;
   // forward
   Split u;

@@ -752,6 +752,201 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ CTA-pair split-K variant
+//
+// One 256 x BN output tile (and one K split, blockIdx.z) per CTA pair, not
+// persistent: the pair-tile operand rate of the kernel above, with the 1-CTA
+// kernel's epilogue interface (a single accumulator, an idle stage ring and an
+// aux barrier after the main loop, split bookkeeping). Epilogues that read the
+// A stages (kReadsA: the norm's sum of squares over W0 rows) cannot wait on
+// the stages' full barrier, which lives in the leader CTA only; instead the
+// leader's MMA thread commits each stage to a "consumed" barrier in both CTAs
+// (the stage's data has been read by the tensor cores, so it is in shared
+// memory), each CTA's epilogue warps read their own 128 A rows there, and the
+// stage returns to that CTA's producer when its four epilogue warps have
+// arrived on its empty barrier.
+
+template <class Cfg, class Epi>
+struct PairSplitLayout {
+  static constexpr int STAGES_RAW = kSmemBudget / Cfg::STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static_assert(STAGES >= 2, "stages");
+  static constexpr int SMEM_BYTES = STAGES * Cfg::STAGE_BYTES + Cfg::BAR_BYTES + 1024;
+};
+
+template <class Cfg, class Epi>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_sm100_pair_split_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tA1,
+                                 const __grid_constant__ CUtensorMap tB0, const __grid_constant__ CUtensorMap tB1,
+                                 const GemmGeom geom, const __grid_constant__ typename Epi::Params ep) {
+  constexpr int STAGES = PairSplitLayout<Cfg, Epi>::STAGES;
+  constexpr bool READS_A = Epi::kReadsA;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* cons = empty + STAGES;  // [STAGES], used when READS_A
+  uint64_t* accf = cons + STAGES;
+  uint64_t* aux = accf + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(aux + 1);
+  static_assert((3 * 8 + 2) * 8 + 8 <= Cfg::BAR_BYTES, "barrier area");
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int n_tiles = (geom.N + Cfg::BN - 1) / Cfg::BN;
+  const int t = blockIdx.x >> 1;
+  const int tm = t / n_tiles, tn = t - tm * n_tiles;
+  const int split = blockIdx.z;
+  const int kb_total = geom.kb0 + geom.kb1;
+  const int kb_begin = split * geom.kb_per_split;
+  const int kb_end = min(kb_total, kb_begin + geom.kb_per_split);
+  const int nkb = kb_end > kb_begin ? kb_end - kb_begin : 0;
+
+  if (threadIdx.x == 0) {
+#pragma unroll 1
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], READS_A ? 4 : 1);
+      mbar_init(&cons[s], 1);
+    }
+    mbar_init(accf, 1);
+    mbar_init(aux, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tA0);
+    prefetch_tmap(&tB0);
+    if (geom.kb1 > 0) {
+      prefetch_tmap(&tA1);
+      prefetch_tmap(&tB1);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, Cfg::ACC_COLS);  // one accumulator: one tile per pair
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_trigger();
+  pdl_wait();
+
+  const int m0 = tm * 2 * kBM + (int)rank * kBM;
+  if (warp == 0) {
+    if (lane == 0) {
+      const int nb0 = tn * Cfg::BN + (int)rank * Cfg::H0;
+      const int nb1 = tn * Cfg::BN + Cfg::N0 + (int)rank * Cfg::H1;
+#pragma unroll 1
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % STAGES;
+        if (!mbar_wait(&empty[s], ((uint32_t)(i / STAGES) & 1u) ^ 1u)) break;
+        uint8_t* sa = smem + s * Cfg::STAGE_BYTES;
+        uint8_t* sb = sa + Cfg::A_BYTES;
+        const uint32_t fb = mapa_shared(smem_u32(&full[s]), 0);
+        if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
+        const int kb = kb_begin + i;
+        const bool src1 = kb >= geom.kb0;
+        const int k0 = (src1 ? kb - geom.kb0 : kb) * kBK;
+        const int k0a = (src1 && geom.a1_kwrap > 0) ? k0 % geom.a1_kwrap : k0;
+        const CUtensorMap* ta = src1 ? &tA1 : &tA0;
+        const CUtensorMap* tb = src1 ? &tB1 : &tB0;
+        if (!Cfg::A_MN) {
+          tma_load_2d_pair(sa, ta, fb, k0a, m0);
+        } else {
+          tma_load_2d_pair(sa, ta, fb, m0, k0a);
+          tma_load_2d_pair(sa + 8192, ta, fb, m0 + 64, k0a);
+        }
+#pragma unroll
+        for (int j = 0; j < Cfg::B0_LOADS; ++j) {
+          if (!Cfg::B_MN)
+            tma_load_2d_pair(sb + j * Cfg::B_BOX * 128, tb, fb, k0, nb0 + j * Cfg::B_BOX);
+          else
+            tma_load_2d_pair(sb + j * 8192, tb, fb, nb0 + j * 64, k0);
+        }
+#pragma unroll
+        for (int j = 0; j < Cfg::B1_LOADS; ++j) {
+          if (!Cfg::B_MN)
+            tma_load_2d_pair(sb + Cfg::B1_OFFSET + j * Cfg::B_BOX * 128, tb, fb, k0, nb1 + j * Cfg::B_BOX);
+          else
+            tma_load_2d_pair(sb + Cfg::B1_OFFSET + j * 8192, tb, fb, nb1 + j * 64, k0);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc0 = idesc_bf16_f32(2 * kBM, Cfg::N0, Cfg::A_MN, Cfg::B_MN);
+      constexpr uint32_t idesc1 = idesc_bf16_f32(2 * kBM, Cfg::N1 > 0 ? Cfg::N1 : 16, Cfg::A_MN, Cfg::B_MN);
+      constexpr uint32_t a_kstep = Cfg::A_MN ? 2048u : 32u;
+      constexpr uint32_t b_kstep = Cfg::B_MN ? 2048u : 32u;
+      constexpr uint32_t a_lbo = Cfg::A_MN ? 8192u : 16u;
+      constexpr uint32_t b_lbo = Cfg::B_MN ? 8192u : 16u;
+#pragma unroll 1
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % STAGES;
+        if (!mbar_wait(&full[s], (uint32_t)(i / STAGES) & 1u)) break;
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + s * Cfg::STAGE_BYTES);
+        const uint32_t sb = sa + Cfg::A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(sa + kk * a_kstep, a_lbo, 1024u);
+          const uint64_t bd0 = sdesc_sw128(sb + kk * b_kstep, b_lbo, 1024u);
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+          umma_bf16_pair(tmem, ad, bd0, idesc0, acc);
+          if (Cfg::N1 > 0) {
+            const uint64_t bd1 = sdesc_sw128(sb + Cfg::B1_OFFSET + kk * b_kstep, b_lbo, 1024u);
+            umma_bf16_pair(tmem + (uint32_t)Cfg::N0, ad, bd1, idesc1, acc);
+          }
+        }
+        umma_commit_pair(READS_A ? &cons[s] : &empty[s], 0x3);
+      }
+      umma_commit_pair(accf, 0x3);
+    }
+  } else {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    typename Epi::RowState st{};
+    if (READS_A) {
+#pragma unroll 1
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % STAGES;
+        if (!mbar_wait(&cons[s], (uint32_t)(i / STAGES) & 1u)) break;
+        Epi::on_a_stage(ep, st, smem + s * Cfg::STAGE_BYTES + row * 128, kb_begin + i >= geom.kb0);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
+    }
+    mbar_wait(accf, 0);
+    tc_fence_after();
+    EpiCtx c;
+    c.taddr = tmem + ((uint32_t)(q * 32) << 16);
+    c.row = row;
+    c.m = m0 + row;
+    c.n0 = tn * Cfg::BN;
+    c.split = split;
+    c.has_acc = nkb > 0;
+    c.stage_smem = smem;
+    c.stage_bytes = STAGES * Cfg::STAGE_BYTES;
+    c.aux_bar = aux;
+    c.tA1 = &tA1;
+    c.tile_id = (tm * 2 + (int)rank) * n_tiles + tn;
+    c.splits = (int)gridDim.z;
+    c.flag = tmem_slot + 1;
+    Epi::template run<Cfg::BN>(ep, st, c, geom);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, Cfg::ACC_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ epilogues
 
 __device__ __forceinline__ void store_bf16x8(__nv_bfloat16* dst, const float* v) {
