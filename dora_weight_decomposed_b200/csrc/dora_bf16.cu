@@ -189,43 +189,6 @@ static cudaError_t launch_gemm(const GemmArgs& g, const typename Epi::Params& ep
 }
 
 // Persistent launch: one CTA per SM (at most one per tile), no K split.
-template <class Cfg, class Epi>
-static cudaError_t launch_gemm_persistent(const GemmArgs& g, const typename Epi::Params& ep, int sms,
-                                          cudaStream_t st) {
-  CUtensorMap ta0, ta1, tb0, tb1;
-  const int a_box = Cfg::A_MN ? 64 : kBM;
-  const int b_box = Cfg::B_MN ? 64 : Cfg::B_BOX;
-  t_detail.clear();
-  if (!make_map(&ta0, g.a0, a_box, "A source 0") || !make_map(&tb0, g.b0, b_box, "B source 0"))
-    return cudaErrorInvalidValue;
-  const int kb0 = (int)ceil_div(g.K0, kBK);
-  const int kb1 = g.K1 > 0 ? (int)ceil_div(g.K1, kBK) : 0;
-  if (kb1 > 0) {
-    if (!make_map(&ta1, g.a1, a_box, "A source 1") || !make_map(&tb1, g.b1, b_box, "B source 1"))
-      return cudaErrorInvalidValue;
-  } else {
-    ta1 = ta0;
-    tb1 = tb0;
-  }
-  GemmGeom geom{g.M, g.N, kb0, kb1, kb0 + kb1, g.a1_kwrap};
-  const long long tiles = ceil_div(g.N, Cfg::BN) * ceil_div(g.M, kBM);
-  const unsigned grid = (unsigned)std::max<long long>(1, std::min<long long>(tiles, sms));
-  auto kern = gemm_sm100_persistent_kernel<Cfg, Epi>;
-  static std::atomic<unsigned long long> smem_set{0};
-  cudaError_t e = set_smem_once(smem_set, kern, Cfg::SMEM_BYTES);
-  if (e != cudaSuccess) {
-    t_detail = "shared-memory attribute (" + std::to_string(Cfg::SMEM_BYTES) + " bytes)";
-    return e;
-  }
-  {
-    ProfRange pr(g.name, st);
-    e = launch_pdl(kern, dim3(grid), dim3(kGemmThreads), Cfg::SMEM_BYTES, st, ta0, ta1, tb0, tb1, geom, ep);
-  }
-  if (e == cudaSuccess) e = cudaGetLastError();
-  if (e != cudaSuccess) t_detail = "persistent launch grid " + std::to_string(grid);
-  return e;
-}
-
 // CTA-pair persistent launch: clusters of two CTAs, one pair per two SMs.
 template <class Cfg, class Epi>
 static cudaError_t launch_gemm_pair(const GemmArgs& g, const typename Epi::Params& ep, int sms, cudaStream_t st) {

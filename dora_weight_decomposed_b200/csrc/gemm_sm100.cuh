@@ -291,14 +291,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-// ------------------------------------------------------------------ persistent variant
+// ------------------------------------------------------------------ tile order
 //
-// One CTA per SM walks the output tiles t = blockIdx.x, blockIdx.x + gridDim.x, ...
-// in groups of kGroupM m-tiles (m fastest inside a group), so the tiles in
-// flight at one time share their A rows and B columns in L2. TMEM holds two
-// 256-column accumulators: while the epilogue warps drain tile j from one, the
-// MMA warp fills the other with tile j + 1. The shared-memory ring runs on
-// across tiles. No K split; the epilogue may not read A stages.
+// Persistent kernels walk the output tiles t = first, first + step, ... in
+// groups of kGroupM m-tiles (m fastest inside a group), so the tiles in flight
+// at one time share their A rows and B columns in L2.
 constexpr int kGroupM = 8;
 
 __device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int& m, int& n) {
@@ -309,184 +306,6 @@ __device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int
   const int rem = t - grp * per_group;
   m = first_m + rem % gm;
   n = rem / gm;
-}
-
-template <class Cfg, class Epi>
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_sm100_persistent_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tA1,
-                                 const __grid_constant__ CUtensorMap tB0, const __grid_constant__ CUtensorMap tB1,
-                                 const GemmGeom geom, const typename Epi::Params ep) {
-  static_assert(Cfg::BN <= 256, "two accumulators must fit in 512 TMEM columns");
-  static_assert(!Epi::kReadsA, "persistent epilogues do not read A stages");
-  constexpr int STAGES = Cfg::STAGES;
-  constexpr uint32_t ACC_COLS = Cfg::BN <= 32 ? 32 : Cfg::BN <= 64 ? 64 : Cfg::BN <= 128 ? 128 : 256;
-  constexpr uint32_t TMEM_COLS = 2 * ACC_COLS < 32 ? 32 : 2 * ACC_COLS;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
-  uint64_t* empty = full + STAGES;
-  uint64_t* accf = empty + STAGES;  // [2]
-  uint64_t* acce = accf + 2;        // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int m_tiles = (geom.M + kBM - 1) / kBM;
-  const int n_tiles = (geom.N + Cfg::BN - 1) / Cfg::BN;
-  const int tiles = m_tiles * n_tiles;
-  const int nkb = geom.kb0 + geom.kb1;
-
-  if (threadIdx.x == 0) {
-#pragma unroll 1
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&accf[b], 1);
-      mbar_init(&acce[b], 4);
-    }
-    fence_mbar_init();
-  }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tA0);
-    prefetch_tmap(&tB0);
-    if (geom.kb1 > 0) {
-      prefetch_tmap(&tA1);
-      prefetch_tmap(&tB1);
-    }
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  pdl_trigger();
-  pdl_wait();
-
-  if (warp == 0) {
-    if (lane == 0) {
-      int it = 0;
-      bool ok = true;
-#pragma unroll 1
-      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-        int m_tile, n_tile;
-        tile_coords(t, m_tiles, n_tiles, m_tile, n_tile);
-        const int m0 = m_tile * kBM;
-        const int n0 = n_tile * Cfg::BN;
-#pragma unroll 1
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!mbar_wait(&empty[s], ph ^ 1u)) {
-            ok = false;
-            break;
-          }
-          uint8_t* sa = smem + s * Cfg::STAGE_BYTES;
-          uint8_t* sb = sa + Cfg::A_BYTES;
-          mbar_arrive_expect_tx(&full[s], Cfg::STAGE_BYTES);
-          const bool src1 = kb >= geom.kb0;
-          const int k0 = (src1 ? kb - geom.kb0 : kb) * kBK;
-          const int k0a = (src1 && geom.a1_kwrap > 0) ? k0 % geom.a1_kwrap : k0;
-          const CUtensorMap* ta = src1 ? &tA1 : &tA0;
-          const CUtensorMap* tb = src1 ? &tB1 : &tB0;
-          if (!Cfg::A_MN) {
-            tma_load_2d(sa, ta, &full[s], k0a, m0);
-          } else {
-            tma_load_2d(sa, ta, &full[s], m0, k0a);
-            tma_load_2d(sa + 8192, ta, &full[s], m0 + 64, k0a);
-          }
-#pragma unroll
-          for (int j = 0; j < Cfg::B_LOADS; ++j) {
-            if (!Cfg::B_MN)
-              tma_load_2d(sb + j * Cfg::B_BOX * 128, tb, &full[s], k0, n0 + j * Cfg::B_BOX);
-            else
-              tma_load_2d(sb + j * 8192, tb, &full[s], n0 + j * 64, k0);
-          }
-        }
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kBM, Cfg::BN, Cfg::A_MN, Cfg::B_MN);
-      constexpr uint32_t a_kstep = Cfg::A_MN ? 2048u : 32u;
-      constexpr uint32_t b_kstep = Cfg::B_MN ? 2048u : 32u;
-      constexpr uint32_t a_lbo = Cfg::A_MN ? 8192u : 16u;
-      constexpr uint32_t b_lbo = Cfg::B_MN ? 8192u : 16u;
-      int it = 0, j = 0;
-      bool ok = true;
-#pragma unroll 1
-      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++j) {
-        const int b = j & 1;
-        const uint32_t uph = (uint32_t)(j >> 1) & 1u;
-        if (!mbar_wait(&acce[b], uph ^ 1u)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + (uint32_t)b * ACC_COLS;
-#pragma unroll 1
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!mbar_wait(&full[s], ph)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sa = smem_u32(smem + s * Cfg::STAGE_BYTES);
-          const uint32_t sb = sa + Cfg::A_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(sa + kk * a_kstep, a_lbo, 1024u);
-            const uint64_t bd = sdesc_sw128(sb + kk * b_kstep, b_lbo, 1024u);
-            umma_bf16(d_tmem, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-          }
-          umma_commit(&empty[s]);
-        }
-        umma_commit(&accf[b]);
-      }
-    }
-  } else {
-    const int q = warp & 3;
-    const int row = q * 32 + lane;
-    typename Epi::RowState st{};
-    int j = 0;
-#pragma unroll 1
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
-      const int b = j & 1;
-      const uint32_t uph = (uint32_t)(j >> 1) & 1u;
-      if (!mbar_wait(&accf[b], uph)) break;
-      tc_fence_after();
-      int m_tile, n_tile;
-      tile_coords(t, m_tiles, n_tiles, m_tile, n_tile);
-      EpiCtx c;
-      c.taddr = tmem + (uint32_t)b * ACC_COLS + ((uint32_t)(q * 32) << 16);
-      c.row = row;
-      c.m = m_tile * kBM + row;
-      c.n0 = n_tile * Cfg::BN;
-      c.split = 0;
-      c.has_acc = nkb > 0;
-      c.stage_smem = nullptr;
-      c.stage_bytes = 0;
-      c.aux_bar = nullptr;
-      c.tA1 = &tA1;
-      c.tile_id = t;
-      c.splits = 1;
-      c.flag = nullptr;
-      Epi::template run<Cfg::BN>(ep, st, c, geom);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acce[b]);
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
-  }
 }
 
 // ------------------------------------------------------------------ CTA-pair persistent variant
