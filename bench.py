@@ -634,6 +634,7 @@ def main(argv=None):
            "timing": "CUDA graphs per call, CUDA events per step, max over ranks"}
     if args.impl == "reference":
         cfg["timing"] = "wall clock over the CPU oracle steps"
+        cfg["l2"] = "not applicable (host CPU)"
         return run_reference(args, wl, cfg)
     return run_ours(args, wl, cfg)
 
