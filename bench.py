@@ -59,7 +59,7 @@ def parse_args(argv=None):
     ap.add_argument("--ref-tokens", type=int, default=256, help="tokens per reference-arm step")
     ap.add_argument("--ref-rows", type=int, default=1024, help="output rows per reference-arm step")
     ap.add_argument("--no-merge", action="store_true",
-                    help="skip the inference, full-gradient and deployment-merge measurements")
+                    help="skip the inference, full-gradient, DVoRA and deployment-merge measurements")
     return ap.parse_args(argv)
 
 
@@ -567,6 +567,34 @@ def run_ours(args, wl, cfg):
                     "api": "dora_backward_full", "l2": "flushed before every call"}
         del gf, wsf
 
+    # ---- DVoRA's extra calls on the same layer: form B' = diag(b) B diag(d), and db, dd from dB'
+    vera = None
+    if rank == 0 and not args.no_merge:
+        bv = torch.linspace(0.5, 1.5, do, device=dev)
+        dv = torch.linspace(-1.0, 1.0, r, device=dev)
+        Bp = torch.empty_like(B)
+        wsv = torch.empty(max(dw.dora_workspace_size(do, 8, r, bf, 1.0, 0, dw.DORA_OP_VERA_GRAD), 256),
+                          dtype=torch.uint8, device=dev)
+        timings = {}
+        for name, fn in (("compose", lambda: dw.dora_vera_compose(B, bv, dv, out=Bp)),
+                         ("grad", lambda: dw.dora_vera_grad(B, bv, dv, dB, ws=wsv))):
+            fn()
+            vev = []
+            for i in range(max(3, args.warmup) + 20):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                if i >= max(3, args.warmup):
+                    vev.append((e0, e1))
+            torch.cuda.synchronize()
+            timings[name] = statistics.median(a.elapsed_time(b_) for a, b_ in vev)
+        vb = {"compose": 2 * (2 * do * r) + 4 * (do + r), "grad": 2 * (2 * do * r) + 8 * (do + r)}
+        vera = {k: {"us": timings[k] * 1e3, "gbs": vb[k] / (timings[k] * 1e-3) / 1e9} for k in timings}
+        vera["api"] = "dora_vera_compose, dora_vera_grad ([d_out x r] passes; launch-latency scale)"
+        del Bp, wsv
+
     # ---- deployment merge W' = diag(g) (W0 + s B A) on the same layer (not part of the step)
     merge = None
     if rank == 0 and not args.no_merge:
@@ -616,6 +644,7 @@ def run_ours(args, wl, cfg):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
             "norm_tflops": norm_flops / (phase_ms["norm"] * 1e-3) / 1e12, "phase_ms": phase_ms,
             "roofline": roof, "kernels": kernels, "inference": infer, "backward_full": full_bwd, "merge": merge,
+            "dvora": vera,
             "gpu_launches": int(launches_per_step * args.steps),
             "clocks": clocks.summary(), "e2e": e2e, "cpu_baseline": cpu, "device_status": status,
             "step_ms_min": min(step_ms), "step_ms_median": statistics.median(step_ms)}

@@ -132,3 +132,22 @@ def test_side_stream_and_no_dx():
     tl.check_tensor("y", y, ref["y"], "bf16")
     tl.check_tensor("dA", dA, ref["dA"], "bf16")
     tl.check_tensor("dm", dm, ref["dm"], "bf16")
+
+
+def test_zero_norm_row_propagates():
+    """A row with W0_i = 0 and B_i = 0 has C_i = 0 (no epsilon, read 5 of the design notes): g_i and
+    g_i - 1 are +inf for m_i > 0 and the row's outputs are NaN (inf * 0), as in the oracle; the other
+    rows are unaffected."""
+    wl = workload("c2", d_out=128, d_in=256, T=40)
+    inp = make_inputs(wl)
+    inp["W0"][5] = 0.0
+    inp["B"][5] = 0.0
+    dev = tl.to_device(inp)
+    out = tl.run_gpu(dev, wl.s)
+    C, g, gm1, y = (tl.host(out[k]) for k in ("C", "g", "gm1", "y"))
+    assert C[5] == 0.0 and np.isposinf(g[5]) and np.isposinf(gm1[5])
+    assert np.all(np.isnan(y[:, 5]))
+    ref = tl.run_oracle(inp)
+    keep = np.arange(wl.d_out) != 5
+    assert np.max(np.abs(C[keep] - ref["C"][keep]) / ref["C"][keep]) <= tl.NORM_RTOL
+    tl.check_tensor("y (other rows)", out["y"][:, torch.from_numpy(keep).cuda()], ref["y"][:, keep], "bf16")
