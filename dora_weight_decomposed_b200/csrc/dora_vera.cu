@@ -18,36 +18,74 @@ namespace {
 
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-__device__ __forceinline__ float to_f(float v) { return v; }
-__device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+// V elements of one row per access: 16 bytes for bf16 (whose rows are
+// 16-byte aligned: r is a multiple of 8 and the tensors 16-byte aligned), one
+// element for fp32 (only 4-byte alignment is required there).
 template <class T>
-__device__ __forceinline__ T from_f(float v);
+struct Vec;
 template <>
-__device__ __forceinline__ float from_f<float>(float v) { return v; }
+struct Vec<__nv_bfloat16> {
+  static constexpr int V = 8;
+  __device__ static void load(const __nv_bfloat16* p, float* f) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 t = __bfloat1622float2(h[i]);
+      f[2 * i] = t.x;
+      f[2 * i + 1] = t.y;
+    }
+  }
+  __device__ static void store(__nv_bfloat16* p, const float* f) {
+    uint4 u;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    *reinterpret_cast<uint4*>(p) = u;
+  }
+};
 template <>
-__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+struct Vec<float> {
+  static constexpr int V = 1;
+  __device__ static void load(const float* p, float* f) { f[0] = *p; }
+  __device__ static void store(float* p, const float* f) { *p = f[0]; }
+};
 
 template <class T>
 __global__ void vera_compose_kernel(const T* __restrict__ Bs, const float* __restrict__ b,
                                     const float* __restrict__ d, int d_out, int r, T* __restrict__ Bp) {
-  const long long total = (long long)d_out * r;
+  constexpr int V = Vec<T>::V;
+  const int q = r / V;
+  const long long total = (long long)d_out * q;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
-    const int n = (int)(i / r), c = (int)(i % r);
-    Bp[i] = from_f<T>(b[n] * to_f(Bs[i]) * d[c]);
+    const int n = (int)(i / q), c = (int)(i % q) * V;
+    const long long off = (long long)n * r + c;
+    float f[V];
+    Vec<T>::load(Bs + off, f);
+    const float bn = b[n];
+#pragma unroll
+    for (int j = 0; j < V; ++j) f[j] = bn * f[j] * d[c + j];
+    Vec<T>::store(Bp + off, f);
   }
 }
 
+// One warp per row, V columns per lane and step.
 template <class T>
 __global__ void vera_db_kernel(const T* __restrict__ dBp, const T* __restrict__ Bs, const float* __restrict__ d,
                                int d_out, int r, float* __restrict__ db) {
+  constexpr int V = Vec<T>::V;
   const int warps = blockDim.x / 32;
   const int lane = threadIdx.x & 31;
   for (int n = blockIdx.x * warps + (threadIdx.x >> 5); n < d_out; n += gridDim.x * warps) {
     float acc = 0.f;
-    for (int c = lane; c < r; c += 32) {
+    for (int c = lane * V; c < r; c += 32 * V) {
       const long long i = (long long)n * r + c;
-      acc = fmaf(to_f(dBp[i]) * to_f(Bs[i]), d[c], acc);
+      float g[V], w[V];
+      Vec<T>::load(dBp + i, g);
+      Vec<T>::load(Bs + i, w);
+#pragma unroll
+      for (int j = 0; j < V; ++j) acc = fmaf(g[j] * w[j], d[c + j], acc);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -55,19 +93,55 @@ __global__ void vera_db_kernel(const T* __restrict__ dBp, const T* __restrict__ 
   }
 }
 
-// part[blk][c] = sum over rows [blk * rows, (blk + 1) * rows) of dB'[n][c] b[n] Bs[n][c].
+// part[blk][c] = sum over rows [blk * rows, (blk + 1) * rows) of dB'[n][c] b[n] Bs[n][c]: each thread
+// takes V columns of every (blockDim / (r / V))-th row of the block, then the row lanes are summed
+// through shared memory in a fixed order.
 template <class T>
-__global__ void vera_dd_partial_kernel(const T* __restrict__ dBp, const T* __restrict__ Bs,
-                                       const float* __restrict__ b, int d_out, int r, int rows,
-                                       float* __restrict__ part) {
+__global__ void __launch_bounds__(256) vera_dd_partial_kernel(const T* __restrict__ dBp, const T* __restrict__ Bs,
+                                                              const float* __restrict__ b, int d_out, int r,
+                                                              int rows, float* __restrict__ part) {
+  constexpr int V = Vec<T>::V;
+  __shared__ float red[256 * V];
+  const int q = r / V;  // column groups
   const int n0 = blockIdx.x * rows, n1 = min(d_out, n0 + rows);
-  for (int c = threadIdx.x; c < r; c += blockDim.x) {
-    float acc = 0.f;
-    for (int n = n0; n < n1; ++n) {
-      const long long i = (long long)n * r + c;
-      acc = fmaf(to_f(dBp[i]) * to_f(Bs[i]), b[n], acc);
+  if (q > (int)blockDim.x) {
+    // Rows wider than the block (fp32, r > 256): each thread sums whole columns.
+    for (int c = threadIdx.x; c < r; c += blockDim.x) {
+      float acc = 0.f;
+      for (int n = n0; n < n1; ++n) {
+        float g, w;
+        Vec<T>::load(dBp + (long long)n * r + c, &g);
+        Vec<T>::load(Bs + (long long)n * r + c, &w);
+        acc = fmaf(g * w, b[n], acc);
+      }
+      part[(long long)blockIdx.x * r + c] = acc;
     }
-    part[(long long)blockIdx.x * r + c] = acc;
+    return;
+  }
+  const int lanes = (int)blockDim.x / q;  // row lanes, >= 1
+  const int cg = threadIdx.x % q, rl = threadIdx.x / q;
+  float acc[V];
+#pragma unroll
+  for (int j = 0; j < V; ++j) acc[j] = 0.f;
+  if (rl < lanes) {
+    for (int n = n0 + rl; n < n1; n += lanes) {
+      const long long i = (long long)n * r + cg * V;
+      float g[V], w[V];
+      Vec<T>::load(dBp + i, g);
+      Vec<T>::load(Bs + i, w);
+      const float bn = b[n];
+#pragma unroll
+      for (int j = 0; j < V; ++j) acc[j] = fmaf(g[j] * w[j], bn, acc[j]);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < V; ++j) red[threadIdx.x * V + j] = acc[j];
+  __syncthreads();
+  for (int c = threadIdx.x; c < r; c += blockDim.x) {
+    const int g = c / V, j = c % V;
+    float s = 0.f;
+    for (int l = 0; l < lanes; ++l) s += red[(l * q + g) * V + j];
+    part[(long long)blockIdx.x * r + c] = s;
   }
 }
 
@@ -82,7 +156,7 @@ __global__ void vera_dd_final_kernel(const float* __restrict__ part, int nblk, i
 template <class T>
 cudaError_t vera_compose_t(const dora_desc_t& dsc, const void* Bs, const float* b, const float* d, void* Bp,
                            cudaStream_t st) {
-  const long long total = dsc.d_out * dsc.r;
+  const long long total = dsc.d_out * (dsc.r / Vec<T>::V);
   ProfRange pr("vera_compose", st);
   vera_compose_kernel<T><<<(unsigned)std::min<long long>(cdiv(total, 256), 4096), 256, 0, st>>>(
       (const T*)Bs, b, d, (int)dsc.d_out, (int)dsc.r, (T*)Bp);

@@ -68,11 +68,12 @@ def test_dvora_layer_step(key, ov):
     tl.check_tensor("dd", dd, rdd, wl.dtype, what="dvora")
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
-def test_vera_grad_reductions(dtype):
-    """db, dd from a given dB' (fp32 sums of exact input values): tight tolerance."""
+@pytest.mark.parametrize("dtype,r", [("bf16", 136), ("fp32", 136), ("fp32", 324), ("bf16", 512), ("bf16", 8)])
+def test_vera_grad_reductions(dtype, r):
+    """db, dd from a given dB' (fp32 sums of exact input values): tight tolerance. fp32 rows wider
+    than a block (r > 256) take the reduction's per-column branch."""
     rng = np.random.default_rng(9)
-    d_out, r = 1000, 136
+    d_out = 1000
     Bs = rng.standard_normal((d_out, r))
     dB = rng.standard_normal((d_out, r))
     if dtype == "bf16":
