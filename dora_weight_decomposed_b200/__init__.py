@@ -24,6 +24,7 @@ import threading
 
 __all__ = ["DoraError", "load_library", "library_path", "dora_workspace_size", "dora_norm", "dora_forward",
            "dora_norm_noalloc", "dora_backward", "dora_backward_full", "dora_merge", "dora_vera_compose",
+           "dora_selftest_timeout",
            "dora_vera_grad", "dora_device_status", "dora_last_error",
            "dora_version",
            "dora_profile_start",
@@ -37,6 +38,7 @@ STATUS_NAMES = {0: "DORA_OK", 1: "DORA_EINVAL", 2: "DORA_EUNSUPPORTED", 3: "DORA
                 5: "DORA_ETIMEOUT"}
 EXPORTED_SYMBOLS = ("dora_workspace_size", "dora_norm", "dora_norm_noalloc", "dora_forward", "dora_backward",
                     "dora_backward_full", "dora_merge", "dora_vera_compose", "dora_vera_grad", "dora_device_status",
+                    "dora_selftest_timeout",
                     "dora_profile_start", "dora_profile_stop", "dora_profile_count", "dora_profile_read",
                     "dora_last_error", "dora_version")
 
@@ -96,6 +98,8 @@ def load_library() -> ctypes.CDLL:
         lib.dora_vera_grad.restype = ctypes.c_int
         lib.dora_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint)]
         lib.dora_device_status.restype = ctypes.c_int
+        lib.dora_selftest_timeout.argtypes = [ctypes.c_uint32, P, P]
+        lib.dora_selftest_timeout.restype = ctypes.c_int
         lib.dora_profile_start.argtypes = [ctypes.c_int]
         lib.dora_profile_start.restype = ctypes.c_int
         lib.dora_profile_stop.argtypes = []
@@ -283,6 +287,18 @@ def dora_device_status(stream=None) -> int:
     if st not in (0, 5):
         _check(st)
     return int(flags.value)
+
+
+def dora_selftest_timeout(limit_us: int = 20000, stream=None) -> int:
+    """Run the failure-detection self-test kernel (a bounded wait that runs out).
+
+    Returns the word the kernel wrote (1 = its wait ran out); the timeout is
+    also left in the device status word for the next dora_device_status.
+    """
+    torch = _torch()
+    scratch = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _check(load_library().dora_selftest_timeout(int(limit_us), _ptr(scratch), _stream_ptr(stream)))
+    return int(scratch.item())
 
 
 def dora_profile_start(capacity: int = 4096) -> None:

@@ -454,6 +454,15 @@ dora_status_t dora_backward_full(const dora_desc_t* desc, int64_t T, const void*
                        stream);
 }
 
+dora_status_t dora_selftest_timeout(uint32_t limit_us, unsigned int* scratch, dora_stream_t stream) {
+  if (limit_us < 1 || limit_us > 1000000) {
+    set_error("limit_us must be in 1 .. 1000000");
+    return DORA_EINVAL;
+  }
+  if (!check_ptr(scratch, "scratch", 4)) return DORA_EINVAL;
+  return selftest_timeout(limit_us, scratch, reinterpret_cast<cudaStream_t>(stream));
+}
+
 dora_status_t dora_device_status(dora_stream_t stream, unsigned int* flags_out) {
   if (!flags_out) {
     set_error("flags_out is NULL");

@@ -1064,6 +1064,25 @@ dora_status_t bf16_backward_full(const dora_desc_t& d, const Plan& p, int64_t T,
 
 namespace dora {
 
+// Failure-detection self-test: one thread waits, through the same bounded
+// wait every kernel uses, on an mbarrier that nothing ever completes. The wait
+// runs out after limit_ns, records the timeout in this library's device status
+// word and the kernel returns; nothing faults, traps or hangs.
+__global__ void selftest_wait_timeout_kernel(uint64_t limit_ns, unsigned int* waited_out) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    const bool done = mbar_wait(&bar, 0, limit_ns);
+    *waited_out = done ? 0u : 1u;
+  }
+}
+
+dora_status_t selftest_timeout(uint32_t limit_us, unsigned int* scratch, cudaStream_t st) {
+  selftest_wait_timeout_kernel<<<1, 32, 0, st>>>((uint64_t)limit_us * 1000ull, scratch);
+  return cuda_status(cudaGetLastError(), "dora_selftest_timeout");
+}
+
 cudaError_t read_and_clear_device_status(cudaStream_t st, unsigned int* out) {
   cudaError_t e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return e;

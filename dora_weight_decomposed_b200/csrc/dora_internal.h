@@ -66,6 +66,8 @@ void set_error(const std::string& msg);
 
 // Status word written by kernels whose bounded waits ran out.
 cudaError_t read_and_clear_device_status(cudaStream_t st, unsigned int* out);
+// One kernel whose bounded wait runs out after limit_us (failure-detection test).
+dora_status_t selftest_timeout(uint32_t limit_us, unsigned int* scratch, cudaStream_t st);
 
 // bf16 path (tcgen05 / TMA kernels)
 dora_status_t bf16_norm(const dora_desc_t& d, const Plan& p, const void* W0, const void* A, const void* B,

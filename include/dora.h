@@ -224,6 +224,18 @@ DORA_API dora_status_t dora_merge(const dora_desc_t* desc, const void* W0, const
 DORA_API dora_status_t dora_device_status(dora_stream_t stream, unsigned int* flags_out);
 
 /*
+ * dora_selftest_timeout -- exercise the failure detection without a fault.
+ * Launches one kernel on `stream` whose single thread waits, through the same
+ * bounded wait the compute kernels use, on an mbarrier that nothing completes;
+ * after limit_us microseconds (1 .. 1000000) the wait gives up, records the
+ * timeout in the device status word and the kernel returns. The next
+ * dora_device_status on that stream then reports bit 0 and DORA_ETIMEOUT, and
+ * the context stays usable. scratch: one device word the kernel writes (1 =
+ * the wait ran out). Nothing faults, traps or hangs.
+ */
+DORA_API dora_status_t dora_selftest_timeout(uint32_t limit_us, unsigned int* scratch, dora_stream_t stream);
+
+/*
  * Kernel timing (benchmarks and tracing; not part of the compute path).
  * dora_profile_start(capacity) creates 2 * capacity CUDA events and, until
  * dora_profile_stop(), brackets each kernel the library launches with a pair of

@@ -158,3 +158,11 @@ def test_full_backward_validation(lib):
     st = lib.dora_backward_full(ctypes.byref(d), 8, fake, fake, fake, fake, fake, fake, fake, None, fake, fake, fake,
                                 fake, fake, fake, 1 << 30, None)
     assert st == 1 and "su_save" in dw.dora_last_error()
+
+
+def test_selftest_timeout_validation(lib):
+    # Limits outside 1 us .. 1 s and a NULL scratch word are rejected before any launch.
+    fake = ctypes.c_void_p(4096)
+    assert lib.dora_selftest_timeout(0, fake, None) == 1
+    assert lib.dora_selftest_timeout(1000001, fake, None) == 1
+    assert lib.dora_selftest_timeout(1000, None, None) == 1 and "scratch" in dw.dora_last_error()
