@@ -79,6 +79,7 @@ __global__ void vera_db_kernel(const T* __restrict__ dBp, const T* __restrict__ 
   const int lane = threadIdx.x & 31;
   for (int n = blockIdx.x * warps + (threadIdx.x >> 5); n < d_out; n += gridDim.x * warps) {
     float acc = 0.f;
+#pragma unroll 2
     for (int c = lane * V; c < r; c += 32 * V) {
       const long long i = (long long)n * r + c;
       float g[V], w[V];
@@ -124,6 +125,7 @@ __global__ void __launch_bounds__(256) vera_dd_partial_kernel(const T* __restric
 #pragma unroll
   for (int j = 0; j < V; ++j) acc[j] = 0.f;
   if (rl < lanes) {
+#pragma unroll 4
     for (int n = n0 + rl; n < n1; n += lanes) {
       const long long i = (long long)n * r + cg * V;
       float g[V], w[V];
