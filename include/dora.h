@@ -52,7 +52,7 @@ typedef struct CUstream_st* dora_stream_t;
 typedef enum {
   DORA_OK = 0,
   DORA_EINVAL = 1,        /* null pointer, bad size, misalignment, bad dtype      */
-  DORA_EUNSUPPORTED = 2,  /* valid request this build does not serve (r > 512, no sm_100 device) */
+  DORA_EUNSUPPORTED = 2,  /* valid request the library does not serve (r > 512, no sm_100 device) */
   DORA_EWORKSPACE = 3,    /* ws_bytes below dora_workspace_size()                 */
   DORA_ECUDA = 4,         /* a CUDA call or kernel launch failed                  */
   DORA_ETIMEOUT = 5       /* a kernel's bounded wait ran out (see dora_device_status) */
