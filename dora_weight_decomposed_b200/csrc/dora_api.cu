@@ -152,9 +152,11 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
     const double kbB = 64.0 * 2.0;  // bytes per K element pair of rows (x 64 K per k-block)
     if (op == DORA_OP_NORM) {
       // The Gram GEMM (CTA pairs, one tile column) is small: split K over the
-      // pairs, with its fp32 partials capped at 8 MiB.
+      // pairs, with its fp32 partials capped at 8 MiB and at least four
+      // k-blocks per split (the finalize sums the splits one after another).
       p.gram_bn = bn_pair_k(r);
-      const int64_t gram_max = std::max<int64_t>(1, (int64_t(8) << 20) / (r * r * 4));
+      const int64_t gram_max = std::max<int64_t>(
+          1, std::min<int64_t>((int64_t(8) << 20) / (r * r * 4), cdiv(d_in, 64) / 4));
       p.gram = choose_split(cdiv(r, 256), cdiv(d_in, 64), p.sms / 2, kbB * (128 + p.gram_bn / 2.0), 0.0,
                             (double)r * r, gram_max);
       p.off_gram_part = take((size_t)p.gram.splits * r * r * 4);
@@ -199,7 +201,8 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
         p.off_kappa = take((size_t)d_out * 4);
         p.off_bk = take((size_t)d_out * r * 2);
         p.gram_bn = bn_pair_k(r);
-        const int64_t gram_max = std::max<int64_t>(1, (int64_t(8) << 20) / (r * r * 4));
+        const int64_t gram_max = std::max<int64_t>(
+            1, std::min<int64_t>((int64_t(8) << 20) / (r * r * 4), cdiv(d_in, 64) / 4));
         p.gram = choose_split(cdiv(r, 256), cdiv(d_in, 64), p.sms / 2, kbB * (128 + p.gram_bn / 2.0), 0.0,
                               (double)r * r, gram_max);
         p.off_gram_part = take((size_t)p.gram.splits * r * r * 4);
