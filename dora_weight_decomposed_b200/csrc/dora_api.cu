@@ -185,14 +185,6 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
       p.du = du.split;
       if (p.du.splits > 1) p.off_du_part = take((size_t)p.du.splits * T * r * 4);
       p.off_du = take((size_t)T * r * 2);
-      if (r <= kSkinnyMaxRank) {
-        // Small ranks: dB and dA stream dz and x once on CUDA cores, one fp32
-        // partial per 256-token block, summed by the split reduction.
-        p.skinny = true;
-        p.dB.splits = p.dA.splits = skinny_token_blocks(T);
-        p.off_dB_part = take((size_t)p.dB.splits * d_out * r * 4);
-        p.off_dA_part = take((size_t)p.dA.splits * d_in * r * 4);
-      } else {
       const NarrowChoice dB = choose_narrow_1cta(d_out, r, T, true, p.sms);
       p.dB_bn = dB.bn;
       p.dB = dB.split;
@@ -201,7 +193,6 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
       p.dA_bn = dA.bn;
       p.dA = dA.split;
       if (p.dA.splits > 1) p.off_dA_part = take((size_t)p.dA.splits * d_in * r * 4);
-      }
       // counters of the dm column strips, zeroed by one memset per call
       p.zero_bytes = (size_t)cdiv(d_out, 64) * 4;
       p.off_ctr = take(p.zero_bytes);

@@ -921,22 +921,8 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
                                              reinterpret_cast<float*>(ws + p.off_du_part), "du_reduce", p.sms, st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: du");
   }
-  if (p.skinny) {
-    // Small rank: dB = dz^T su and dA^T = x^T du as CUDA-core streams over dz and x.
-    cudaError_t e = skinny_tn(dz, d_out, su, r, Ti, d_out, r, reinterpret_cast<float*>(ws + p.off_dB_part),
-                              "dB_gemm", st);
-    if (e == cudaSuccess)
-      e = reduce_splits(reinterpret_cast<float*>(ws + p.off_dB_part), p.dB, (long long)d_out * r, d_out, r, 1.0f,
-                        reinterpret_cast<__nv_bfloat16*>(dB), r, false, "dB_reduce", st);
-    if (e == cudaSuccess)
-      e = skinny_tn(x, d_in, du, r, Ti, d_in, r, reinterpret_cast<float*>(ws + p.off_dA_part), "dA_gemm", st);
-    if (e == cudaSuccess)
-      e = reduce_splits(reinterpret_cast<float*>(ws + p.off_dA_part), p.dA, (long long)d_in * r, d_in, r, 1.0f,
-                        reinterpret_cast<__nv_bfloat16*>(dA), d_in, true, "dA_reduce", st);
-    if (e != cudaSuccess) return cuda_status(e, "dora_backward: dB, dA (small rank)");
-  }
   // dB = dz^T su  (both token-major: K = T)
-  if (!p.skinny) {
+  {
     GemmArgs a;
     a.a0 = Mat{dz, Ti, d_out, d_out};
     a.b0 = Mat{su, Ti, r, r};
@@ -950,7 +936,7 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: dB");
   }
   // dA^T = x^T du, stored transposed into dA [r x d_in]
-  if (!p.skinny) {
+  {
     GemmArgs a;
     a.a0 = Mat{x, Ti, d_in, d_in};
     a.b0 = Mat{du, Ti, r, r};

@@ -33,7 +33,6 @@ struct Plan {
   int dm_rowblocks = 0;
   Split du, dB, dA;
   int du_bn = 0, dB_bn = 0, dA_bn = 0;
-  bool skinny = false;  // dB and dA on the CUDA-core token contraction (r <= kSkinnyMaxRank)
   size_t off_dz = 0, off_dm_part = 0, off_du_part = 0, off_du = 0, off_dB_part = 0, off_dA_part = 0;
   // full (non-detached) gradient: kappa, kappa-scaled B, Gram, Q = W' A^T, H = s B^T diag(kappa) B
   Split q, h;
@@ -80,14 +79,6 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
                             const void* W0, const void* A, const void* B, const float* C, const float* g,
                             const void* su, const void* pre, float* dm, void* dA, void* dB, void* dx,
                             uint8_t* ws, cudaStream_t st);
-
-// Token contractions out[i][j] = sum_t P[t][i] Q[t][j] (bf16 in) for ranks
-// r <= kSkinnyMaxRank on CUDA cores: fp32 partials part[token block][W][r],
-// one block of skinny_token_blocks(T) per 256 tokens.
-constexpr int kSkinnyMaxRank = 32;
-int skinny_token_blocks(int64_t T);
-cudaError_t skinny_tn(const void* P, int ldp, const void* Q, int ldq, int T, int W, int r, float* part,
-                      const char* name, cudaStream_t st);
 
 dora_status_t bf16_backward_full(const dora_desc_t& d, const Plan& p, int64_t T, const void* dy, const void* x,
                                  const void* W0, const void* A, const void* B, const float* C, const float* g,
