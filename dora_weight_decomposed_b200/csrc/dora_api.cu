@@ -240,8 +240,9 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
     }
   }
   if (op == DORA_OP_VERA_GRAD) {
-    // Enough row blocks (16 rows each, up to 1184) to keep the loads of the dd pass in flight.
-    p.vera_blocks = (int)std::min<int64_t>(cdiv(d_out, 16), 1184);
+    // Row blocks of the dd pass: 64 rows each, at most 296 (two per SM), so the
+    // final per-column sum over the blocks stays short.
+    p.vera_blocks = (int)std::min<int64_t>(cdiv(d_out, 64), 296);
     p.off_f32_a = take((size_t)p.vera_blocks * r * 4);
   }
   p.total = off;
