@@ -48,13 +48,6 @@ struct Plan {
   size_t total = 0;
 };
 
-// Tile widths of the narrow (N = r) GEMMs: the whole rank in one N tile, so
-// the large operand is streamed once. K-major B tiles step in 16s up to 128,
-// then 256 / 384 / 512; MN-major B tiles are whole 64-column swizzle chunks.
-inline int bn_narrow_k(int64_t r) {
-  return r <= 16 ? 16 : r <= 32 ? 32 : r <= 64 ? 64 : r <= 128 ? 128 : r <= 256 ? 256 : r <= 384 ? 384 : 512;
-}
-inline int bn_narrow_mn(int64_t r) { return r <= 64 ? 64 : r <= 128 ? 128 : r <= 256 ? 256 : r <= 384 ? 384 : 512; }
 // Whole-rank tile width for CTA-pair GEMMs with K-major B (widths 64 .. 512).
 inline int bn_pair_k(int64_t r) { return r <= 64 ? 64 : r <= 128 ? 128 : r <= 256 ? 256 : r <= 384 ? 384 : 512; }
 
