@@ -7,8 +7,14 @@
  *     V' = W0 + s * B A,   C_i = ||V'_i|| (one norm per output row),
  *     y  = x (diag(m / C) V')^T
  *
+ * Calls: dora_norm, dora_forward, dora_backward (the layer step);
+ * dora_backward_full (without the norm's detach), dora_merge (deployment
+ * weight), dora_vera_compose / dora_vera_grad (DVoRA); workspace sizing,
+ * device status, a failure-detection self-test and kernel timing.
+ *
  * Sources: "DoRA 阅读笔记" (zhongzhuzhou.org reading notes on DoRA, arXiv
- * 2402.09353) eq. (1), eq. (6), Algorithm 1, eq. (7), eq. (8), section 3.4;
+ * 2402.09353) eq. (1), eq. (6), Algorithm 1, eq. (7), eq. (8), sections 3.4
+ * and 3.5, appendix A;
  * "Scaling DoRA" (gptget.net/papers/2603.22276) English abstract: the row-wise
  * norm of W + sBA, its factored form (base + cross + Gram terms, no dense B A
  * product), and the fused single-pass composition in a form that is stable
