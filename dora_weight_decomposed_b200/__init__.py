@@ -166,6 +166,26 @@ def _shape(t, shape, name):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
+def _args(dtype, device, **spec):
+    """Check every given tensor (name=(tensor, shape, kind)); kind "t" = the layer dtype, "f" = float32.
+
+    The C ABI cannot see shapes or dtypes: a wrong one would make a kernel read
+    or write past a buffer, so every tensor, inputs and caller-supplied outputs
+    alike, is checked here before anything is launched. None entries (optional
+    outputs) are skipped.
+    """
+    torch = _torch()
+    for name, (t, shape, kind) in spec.items():
+        if t is None:
+            continue
+        _shape(t, shape, name)
+        want = dtype if kind == "t" else torch.float32
+        if t.dtype != want:
+            raise TypeError(f"{name} is {t.dtype}, expected {want}")
+        if t.device != device:
+            raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
 def dora_workspace_size(d_out: int, d_in: int, r: int, dtype, s: float, T: int, op: int) -> int:
     d = _desc(d_out, d_in, r, dtype, s)
     return int(load_library().dora_workspace_size(ctypes.byref(d), int(T), int(op)))
@@ -187,11 +207,8 @@ def dora_norm(W0, A, B, m, s: float, *, norm_out=None, g_out=None, gm1_out=None,
     lib = load_library()
     d_out, d_in = W0.shape
     r = A.shape[0]
-    _shape(A, (r, d_in), "A")
-    _shape(B, (d_out, r), "B")
-    _shape(m, (d_out,), "m")
-    if A.dtype != W0.dtype or B.dtype != W0.dtype or m.dtype != torch.float32:
-        raise TypeError("W0, A, B share one dtype; m is float32")
+    _args(W0.dtype, W0.device, A=(A, (r, d_in), "t"), B=(B, (d_out, r), "t"), m=(m, (d_out,), "f"),
+          norm_out=(norm_out, (d_out,), "f"), g_out=(g_out, (d_out,), "f"), gm1_out=(gm1_out, (d_out,), "f"))
     desc = _desc(d_out, d_in, r, W0.dtype, s)
     f32 = dict(dtype=torch.float32, device=W0.device)
     norm_out = torch.empty(d_out, **f32) if norm_out is None else norm_out
@@ -215,16 +232,17 @@ def dora_forward(x, W0, A, B, gm1, s: float, *, save_for_backward: bool = True, 
     T, d_in = x.shape
     d_out = W0.shape[0]
     r = A.shape[0]
-    _shape(W0, (d_out, d_in), "W0")
-    _shape(A, (r, d_in), "A")
-    _shape(B, (d_out, r), "B")
-    _shape(gm1, (d_out,), "gm1")
-    desc = _desc(d_out, d_in, r, W0.dtype, s)
     dev = x.device
+    _args(W0.dtype, dev, x=(x, (T, d_in), "t"), W0=(W0, (d_out, d_in), "t"), A=(A, (r, d_in), "t"),
+          B=(B, (d_out, r), "t"), gm1=(gm1, (d_out,), "f"), y=(y, (T, d_out), "t"),
+          su_save=(su_save, (T, r), "t"), pre_save=(pre_save, (T, d_out), "t"))
+    desc = _desc(d_out, d_in, r, W0.dtype, s)
     y = torch.empty(T, d_out, dtype=x.dtype, device=dev) if y is None else y
     if save_for_backward:
         su_save = torch.empty(T, r, dtype=x.dtype, device=dev) if su_save is None else su_save
         pre_save = torch.empty(T, d_out, dtype=x.dtype, device=dev) if pre_save is None else pre_save
+    else:
+        su_save = pre_save = None
     wsb, nbytes = _workspace(desc, T, DORA_OP_FORWARD, dev, ws)
     _check(lib.dora_forward(ctypes.byref(desc), T, _ptr(x), _ptr(W0), _ptr(A), _ptr(B), _ptr(gm1), _ptr(y),
                             _ptr(su_save), _ptr(pre_save), _ptr(wsb), nbytes, _stream_ptr(stream)))
@@ -243,11 +261,14 @@ def dora_backward(dy, x, W0, A, B, norm, g, su_save, pre_save, s: float, *, need
     T, d_in = x.shape
     d_out = W0.shape[0]
     r = A.shape[0]
-    _shape(dy, (T, d_out), "dy")
-    _shape(su_save, (T, r), "su_save")
-    _shape(pre_save, (T, d_out), "pre_save")
-    desc = _desc(d_out, d_in, r, W0.dtype, s)
     dev = x.device
+    _args(W0.dtype, dev, dy=(dy, (T, d_out), "t"), x=(x, (T, d_in), "t"), W0=(W0, (d_out, d_in), "t"),
+          A=(A, (r, d_in), "t"), B=(B, (d_out, r), "t"), norm=(norm, (d_out,), "f"), g=(g, (d_out,), "f"),
+          su_save=(su_save, (T, r), "t"), pre_save=(pre_save, (T, d_out), "t"), dm=(dm, (d_out,), "f"),
+          dA=(dA, (r, d_in), "t"), dB=(dB, (d_out, r), "t"), dx=(dx if need_dx else None, (T, d_in), "t"))
+    if su_save is None or pre_save is None:
+        raise ValueError("su_save and pre_save (from dora_forward) are required")
+    desc = _desc(d_out, d_in, r, W0.dtype, s)
     dm = torch.empty(d_out, dtype=torch.float32, device=dev) if dm is None else dm
     dA = torch.empty(r, d_in, dtype=x.dtype, device=dev) if dA is None else dA
     dB = torch.empty(d_out, r, dtype=x.dtype, device=dev) if dB is None else dB
@@ -269,9 +290,8 @@ def dora_merge(W0, A, B, g, s: float, *, out=None, ws=None, stream=None):
     lib = load_library()
     d_out, d_in = W0.shape
     r = A.shape[0]
-    _shape(A, (r, d_in), "A")
-    _shape(B, (d_out, r), "B")
-    _shape(g, (d_out,), "g")
+    _args(W0.dtype, W0.device, A=(A, (r, d_in), "t"), B=(B, (d_out, r), "t"), g=(g, (d_out,), "f"),
+          out=(out, (d_out, d_in), "t"))
     desc = _desc(d_out, d_in, r, W0.dtype, s)
     out = torch.empty_like(W0) if out is None else out
     wsb, nbytes = _workspace(desc, 0, DORA_OP_MERGE, W0.device, ws)
@@ -339,9 +359,8 @@ def dora_norm_noalloc(W0, A, B, m, s: float, *, norm_out=None, g_out=None, gm1_o
     fn.restype = ctypes.c_int
     d_out, d_in = W0.shape
     r = A.shape[0]
-    _shape(A, (r, d_in), "A")
-    _shape(B, (d_out, r), "B")
-    _shape(m, (d_out,), "m")
+    _args(W0.dtype, W0.device, A=(A, (r, d_in), "t"), B=(B, (d_out, r), "t"), m=(m, (d_out,), "f"),
+          norm_out=(norm_out, (d_out,), "f"), g_out=(g_out, (d_out,), "f"), gm1_out=(gm1_out, (d_out,), "f"))
     desc = _desc(d_out, d_in, r, W0.dtype, s)
     f32 = dict(dtype=torch.float32, device=W0.device)
     norm_out = torch.empty(d_out, **f32) if norm_out is None else norm_out
@@ -362,10 +381,7 @@ def dora_vera_compose(B_shared, b, d, *, out=None, s: float = 1.0, stream=None):
     torch = _torch()
     lib = load_library()
     d_out, r = B_shared.shape
-    _shape(b, (d_out,), "b")
-    _shape(d, (r,), "d")
-    if b.dtype != torch.float32 or d.dtype != torch.float32:
-        raise TypeError("b and d are float32")
+    _args(B_shared.dtype, B_shared.device, b=(b, (d_out,), "f"), d=(d, (r,), "f"), out=(out, (d_out, r), "t"))
     desc = _desc(d_out, 8, r, B_shared.dtype, s)
     out = torch.empty_like(B_shared) if out is None else out
     _check(lib.dora_vera_compose(ctypes.byref(desc), _ptr(B_shared), _ptr(b), _ptr(d), _ptr(out),
@@ -378,9 +394,7 @@ def dora_vera_grad(B_shared, b, d, dB, *, s: float = 1.0, ws=None, stream=None):
     torch = _torch()
     lib = load_library()
     d_out, r = B_shared.shape
-    _shape(b, (d_out,), "b")
-    _shape(d, (r,), "d")
-    _shape(dB, (d_out, r), "dB")
+    _args(B_shared.dtype, B_shared.device, b=(b, (d_out,), "f"), d=(d, (r,), "f"), dB=(dB, (d_out, r), "t"))
     desc = _desc(d_out, 8, r, B_shared.dtype, s)
     db = torch.empty(d_out, dtype=torch.float32, device=B_shared.device)
     dd = torch.empty(r, dtype=torch.float32, device=B_shared.device)
