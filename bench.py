@@ -28,6 +28,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -103,14 +104,21 @@ KERNEL_SOURCES = {
 }
 
 
+def _code_only(text):
+    """Source text without comments and blank lines: comment edits do not change a kernel."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*$", "", line).rstrip() for line in text.splitlines())
+    return "\n".join(line for line in lines if line.strip())
+
+
 def source_hash(kernel):
     names = KERNEL_SOURCES.get(kernel)
     if names is None:
         return None
     h = hashlib.sha256()
     for n in names:
-        with open(os.path.join(ROOT, "dora_weight_decomposed_b200", "csrc", n), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "dora_weight_decomposed_b200", "csrc", n), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

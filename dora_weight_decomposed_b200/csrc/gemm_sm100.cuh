@@ -17,7 +17,8 @@
 //   warp 1     allocates TMEM; one lane issues tcgen05.mma and commits
 //   warps 2-5  epilogue: warp w owns TMEM lanes 32*(w%4) .. +31 (= tile rows);
 //              an epilogue may also read each A stage (kReadsA) before it is
-//              released, which the norm uses for the row sums of squares.
+//              released (the CTA-pair split kernel below does the same for the
+//              norm's row sums of squares).
 #pragma once
 
 #include "sm100_ptx.cuh"
