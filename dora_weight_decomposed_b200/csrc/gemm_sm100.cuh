@@ -70,14 +70,16 @@ struct EpiCtx {
   int n0;          // first global output column of the tile
   int split;       // blockIdx.z
   bool has_acc;    // false when this split had no k-blocks (accumulator never written)
-  // Non-persistent kernel only: once the accumulator is complete the stage
-  // ring is idle, and an epilogue may refill it through its own barrier.
+  // Non-persistent kernels only (one CTA per tile, or the CTA-pair split
+  // kernel): once the accumulator is complete the stage ring is idle, and an
+  // epilogue may refill it through its own barrier.
   uint8_t* stage_smem;        // start of the stage ring
   int stage_bytes;            // bytes of the ring
   uint64_t* aux_bar;          // spare mbarrier (count 1), phase 0 unused so far
   const CUtensorMap* tA1;     // A-operand source-1 tensor map
-  // K-split bookkeeping (non-persistent kernel): the output tile's index, the
-  // number of splits, and a shared-memory word for the last-split decision.
+  // K-split bookkeeping (non-persistent kernels): the output rows' index (one
+  // per 128-row block), the number of splits, and a shared-memory word for
+  // the last-split decision.
   int tile_id;
   int splits;
   uint32_t* flag;
