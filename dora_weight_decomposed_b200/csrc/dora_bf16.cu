@@ -3,16 +3,19 @@
 // and the small reductions.
 //
 //   dora_norm     Gram G = A A^T (split-K partials -> (s/2) G as bf16 hi + lo), then
-//                 one GEMM  acc = [W0 | B | B] [A | Gs_hi | Gs_lo]^T  whose epilogue forms
-//                 sum_k W0_ik^2 (read from the W0 tiles in shared memory as they
-//                 stream past) + 2 s B_i . acc_i  per row and K split; a finalize
-//                 kernel sums the splits and takes C, g, g - 1.
+//                 one GEMM on CTA pairs  acc = [W0 | B | B] [A | Gs_hi | Gs_lo]^T  whose
+//                 epilogue forms sum_k W0_ik^2 (read from the W0 tiles in shared
+//                 memory once the MMAs consumed them) + 2 s B_i . acc_i  per row and
+//                 K split; the last split of each row block sums the splits and
+//                 takes C, g, g - 1.
 //                 2 s B_i . acc_i = 2 s B_i (W0 A^T)_i + s^2 B_i G B_i^T: the cross
 //                 and Gram terms of the factored norm (Scaling DoRA abstract).
 //   dora_forward  su = s x A^T, then  pre = [x | su] [W0 | B]^T  with the
 //                 compose y = pre + gm1 * pre  in the epilogue (one rounding).
 //   dora_backward dz = g * dy and the dm column sums in one streaming pass;
 //                 du = s dz B, dB = dz^T su, dA = du^T x, dx = [dz | du] [W0 ; A].
+//   dora_backward_full  the above, then the eq. (A.1) corrections of dB and dA.
+//   dora_merge    W' = diag(g) (W0 + s B A) (merge_sm100.cuh).
 #include <algorithm>
 #include <atomic>
 #include <mutex>
