@@ -156,8 +156,11 @@ def _ptr(t) -> int | None:
 
 
 def _stream_ptr(stream) -> int | None:
+    """The CUDA stream handle; the library launches on the current device, so the stream must be on it."""
     torch = _torch()
     s = stream if stream is not None else torch.cuda.current_stream()
+    if s.device.index != torch.cuda.current_device():
+        raise ValueError(f"stream is on {s.device}, but the current device is cuda:{torch.cuda.current_device()}")
     return s.cuda_stream or None
 
 
@@ -175,6 +178,11 @@ def _args(dtype, device, **spec):
     outputs) are skipped.
     """
     torch = _torch()
+    # The library launches every kernel on the current device: tensors on another
+    # device would hand it pointers that device cannot use.
+    if device.type == "cuda" and device.index != torch.cuda.current_device():
+        raise ValueError(f"tensors are on {device}, but the current device is cuda:{torch.cuda.current_device()}; "
+                         f"call under torch.cuda.device({device.index})")
     for name, (t, shape, kind) in spec.items():
         if t is None:
             continue
@@ -389,15 +397,16 @@ def dora_vera_compose(B_shared, b, d, *, out=None, s: float = 1.0, stream=None):
     return out
 
 
-def dora_vera_grad(B_shared, b, d, dB, *, s: float = 1.0, ws=None, stream=None):
+def dora_vera_grad(B_shared, b, d, dB, *, s: float = 1.0, db=None, dd=None, ws=None, stream=None):
     """Gradients (db [d_out], dd [r], float32) of DVoRA's trained vectors from dB' = dL/dB'."""
     torch = _torch()
     lib = load_library()
     d_out, r = B_shared.shape
-    _args(B_shared.dtype, B_shared.device, b=(b, (d_out,), "f"), d=(d, (r,), "f"), dB=(dB, (d_out, r), "t"))
+    _args(B_shared.dtype, B_shared.device, b=(b, (d_out,), "f"), d=(d, (r,), "f"), dB=(dB, (d_out, r), "t"),
+          db=(db, (d_out,), "f"), dd=(dd, (r,), "f"))
     desc = _desc(d_out, 8, r, B_shared.dtype, s)
-    db = torch.empty(d_out, dtype=torch.float32, device=B_shared.device)
-    dd = torch.empty(r, dtype=torch.float32, device=B_shared.device)
+    db = torch.empty(d_out, dtype=torch.float32, device=B_shared.device) if db is None else db
+    dd = torch.empty(r, dtype=torch.float32, device=B_shared.device) if dd is None else dd
     wsb, nbytes = _workspace(desc, 0, DORA_OP_VERA_GRAD, B_shared.device, ws)
     _check(lib.dora_vera_grad(ctypes.byref(desc), _ptr(B_shared), _ptr(b), _ptr(d), _ptr(dB), _ptr(db), _ptr(dd),
                               _ptr(wsb), nbytes, _stream_ptr(stream)))

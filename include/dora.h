@@ -117,9 +117,12 @@ DORA_API dora_status_t dora_norm(const dora_desc_t* desc, const void* W0, const 
  * is rejected with DORA_EUNSUPPORTED before anything is launched.
  * The first call on a device looks up the array's device address with that
  * device current and caches it; make that first call before any stream
- * capture. All calls on a device share the array and leave their contents in
- * it (each call writes every scratch byte before reading it): calls whose
- * kernels may overlap on the GPU race and must be ordered by the caller.
+ * capture. The cached address belongs to the device's current context: after
+ * cudaDeviceReset() the process must load the library again before calling
+ * this function on that device. All calls on a device share the array and
+ * leave their contents in it (each call writes every scratch byte before
+ * reading it): calls whose kernels may overlap on the GPU race and must be
+ * ordered by the caller.
  */
 DORA_API dora_status_t dora_norm_noalloc(const dora_desc_t* desc, const void* W0, const void* A, const void* B,
                                          const float* m, float* norm_out, float* g_out, float* gm1_out,

@@ -39,7 +39,8 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["adapted_direction", "norm", "forward", "backward", "merge", "vera_direction", "vera_gradients"]
+__all__ = ["adapted_direction", "norm", "norm_factored", "forward", "backward", "merge", "vera_direction",
+           "vera_gradients"]
 
 
 def _f64(a) -> np.ndarray:
@@ -68,6 +69,24 @@ def norm(W0, A, B, m, s: float):
     """
     C = _row_norms(adapted_direction(W0, A, B, s))
     m = _f64(m)
+    return C, m / C, (m - C) / C
+
+
+def norm_factored(W0, A, B, m, s: float):
+    """The same (C, g, g - 1) as norm(), from the factored row norm without the dense B A.
+
+    [Scaling DoRA] abstract: ||W + sBA||_row^2 splits into a base term ||W0_i||^2,
+    a cross term 2 s B_i . (W0 A^T)_i and a Gram term s^2 B_i (A A^T) B_i^T, so
+    only [d_out x r] and [r x r] intermediates are formed. Used as the CPU
+    float64 timing baseline of the factored form (the benchmark times it beside
+    the dense definition); the pins check it against norm().
+    """
+    W0, A, B, m = _f64(W0), _f64(A), _f64(B), _f64(m)
+    s = float(s)
+    base = np.einsum("ij,ij->i", W0, W0)
+    cross = 2.0 * s * np.einsum("ir,ir->i", B, W0 @ A.T)
+    gram = s * s * np.einsum("ir,ir->i", B @ (A @ A.T), B)
+    C = np.sqrt(np.maximum(base + cross + gram, 0.0))
     return C, m / C, (m - C) / C
 
 

@@ -32,6 +32,6 @@ def test_bounded_wait_times_out_and_context_survives():
     wl = workload("c2", d_out=256, d_in=384, T=64)
     inp = tl.prepare(wl)
     out = tl.run_gpu(tl.to_device(inp), wl.s)
-    tl.check_all(out, tl.run_oracle(inp), wl.dtype, what="after a timeout")
+    tl.check_all(out, tl.run_oracle(inp), inp, what="after a timeout")
     assert dw.dora_device_status() == 0
 

@@ -34,20 +34,29 @@ def test_cached_norm_forward_over_batches(key, ov):
     wl = workload(key, **ov)
     inp = tl.prepare(wl, with_backward=False)
     dev = tl.to_device(inp)
-    _, _, gm1 = dw.dora_norm(dev["W0"], dev["A"], dev["B"], dev["m"], wl.s)
+    C, g, gm1 = dw.dora_norm(dev["W0"], dev["A"], dev["B"], dev["m"], wl.s)
+    norm_gpu = {"C": C, "g": g, "gm1": gm1}
+    Cr, gr, gm1r = oracle.norm(inp["W0"], inp["A"], inp["B"], inp["m"], wl.s)
     ws = torch.empty(dw.dora_workspace_size(wl.d_out, wl.d_in, wl.r, torch.bfloat16, wl.s, 300,
                                             dw.DORA_OP_FORWARD), dtype=torch.uint8, device="cuda")
     for seed, T in ((11, 300), (12, 1), (13, 129)):
         x_np = make_inputs(workload(key, **dict(ov, T=T)), with_backward=False, token_seed=seed)["x"]
         x = torch.from_numpy(x_np).cuda().to(torch.bfloat16).contiguous()
-        y, su, pre = dw.dora_forward(x, dev["W0"], dev["A"], dev["B"], gm1, wl.s, save_for_backward=False, ws=ws)
+        y, su, pre = dw.dora_forward(x, dev["W0"], dev["A"], dev["B"], gm1, wl.s, save_for_backward=False, ws=ws,
+                                     y=tl.poisoned((T, wl.d_out), torch.bfloat16))
         assert su is None and pre is None
-        ref = oracle.forward(x_np, inp["W0"], inp["A"], inp["B"], inp["m"], wl.s)
-        tl.check_tensor("y", y, ref, "bf16", what=f"{key} T={T}")
+        ref = {"C": Cr, "g": gr, "gm1": gm1r, "y": oracle.forward(x_np, inp["W0"], inp["A"], inp["B"], inp["m"], wl.s)}
+        batch = dict(inp, x=x_np)
+        what = f"{key} T={T}"
+        tl.check_tensor("y", y, ref["y"], "bf16", what=what)
+        tl.check_rows("y", y, ref["y"], "bf16", what=what)
+        tl.check_elementwise("y", y, ref["y"], tl.element_bounds(batch, ref, norm_gpu, "bf16")["y"], what=what)
         if wl.m_lo is None:  # near-unity layer: the adapted part y - x W0^T must survive too
             base = x_np.astype(np.float64) @ inp["W0"].astype(np.float64).T
-            a, b = tl.host(y) - base, ref - base
+            a, b = tl.host(y) - base, ref["y"] - base
             assert tl.rel_fro(a, b) <= tl.BF16_RTOL and tl.cosine(a, b) >= 0.999, (key, T)
+            if T >= 100:
+                tl.check_near_unity(y, batch, ref, what=what)
 
 
 def test_forward_without_saves_matches_forward_with_saves():

@@ -44,7 +44,7 @@ def _merge_case(wl, rows=None):
     inp = tl.prepare(wl, with_backward=False)
     dev = tl.to_device(inp)
     _, g, _ = dw.dora_norm(dev["W0"], dev["A"], dev["B"], dev["m"], wl.s)
-    Wm = dw.dora_merge(dev["W0"], dev["A"], dev["B"], g, wl.s)
+    Wm = dw.dora_merge(dev["W0"], dev["A"], dev["B"], g, wl.s, out=tl.poisoned(dev["W0"].shape, dev["W0"].dtype))
     W0, A, B, m = inp["W0"], inp["A"], inp["B"], inp["m"]
     if rows is None:
         ref = oracle.merge(W0, A, B, m, wl.s)

@@ -9,6 +9,9 @@ What pins what:
               every output including the full gradient and the merge
   factored    the oracle's dense norm equals base + cross + Gram
               (Scaling DoRA abstract) on random inputs
+  factored_norm  norm_factored (the factored form without the dense B A) gives
+              the dense norm's C, g, g - 1, the golden values, and
+              C = |W0_i| at B = 0 (numpy.linalg.norm)
   zero_B      B = 0 gives C = |W0_i| and g = m / |W0_i| (numpy.linalg.norm)
   init        B = 0 and m = |W0_i| gives y = x W0^T (DoRA notes sec. 3.1:
               training starts from the pretrained weight)
@@ -97,6 +100,24 @@ def pin_factored(orc):
         gram = s * s * np.einsum("ir,rq,iq->i", B, A @ A.T, B)
         C, _, _ = orc.norm(W0, A, B, L["m"], s)
         _close(C * C, base + cross + gram, 1e-12, "factored identity")
+
+
+def pin_factored_norm(orc):
+    rng = np.random.default_rng(8)
+    for (d_out, d_in, r, s) in [(5, 7, 3, 1.3), (16, 40, 8, -0.6), (9, 4, 12, 2.0)]:
+        L = _rand_layer(rng, d_out, d_in, r, 2, s=s)
+        got = orc.norm_factored(L["W0"], L["A"], L["B"], L["m"], s)
+        want = orc.norm(L["W0"], L["A"], L["B"], L["m"], s)
+        for a, b, what in zip(got, want, ("C", "g", "gm1")):
+            _close(a, b, 1e-12, f"factored {what}")
+    for ex in _golden():
+        W0, A, B, m = (np.array(ex[k], dtype=np.float64) for k in ("W0", "A", "B", "m"))
+        C, g, gm1 = orc.norm_factored(W0, A, B, m, float(ex["s"]))
+        _close(C, ex["expected"]["C"], 1e-14, "factored C (golden)")
+        _close(gm1, ex["expected"]["gm1"], 1e-14, "factored gm1 (golden)")
+    L = _rand_layer(rng, 6, 9, 3, 2)
+    C, _, _ = orc.norm_factored(L["W0"], L["A"], np.zeros_like(L["B"]), L["m"], L["s"])
+    _close(C, np.linalg.norm(L["W0"], axis=1), 1e-14, "factored C(B=0)")
 
 
 def pin_zero_B(orc):
@@ -247,7 +268,7 @@ def pin_vera_unit(orc):
     _close(Bp[:, 1] / Bs[:, 1], b * d[1], 1e-15, "column 1 scaled by b d_1")
 
 
-PINS = [pin_golden, pin_factored, pin_zero_B, pin_init, pin_scale, pin_merge, pin_fd_x_m,
+PINS = [pin_golden, pin_factored, pin_factored_norm, pin_zero_B, pin_init, pin_scale, pin_merge, pin_fd_x_m,
         pin_fd_detached, pin_fd_full, pin_a2_term, pin_eq8, pin_near_unity, pin_vera_fd, pin_vera_unit]
 
 
@@ -301,6 +322,7 @@ def test_near_unity_generator():
 
 def _mutant(**overrides):
     ns = types.SimpleNamespace(adapted_direction=oracle.adapted_direction, norm=oracle.norm,
+                               norm_factored=oracle.norm_factored,
                                forward=oracle.forward, backward=oracle.backward, merge=oracle.merge,
                                vera_direction=oracle.vera_direction, vera_gradients=oracle.vera_gradients)
     for k, v in overrides.items():
@@ -361,6 +383,14 @@ def _forward_ignores_C(x, W0, A, B, m, s, C=None):
     return oracle.forward(x, W0, A, B, m, s)
 
 
+def _factored_gram_s(W0, A, B, m, s):
+    """The Gram term scaled by s instead of s^2."""
+    W0, A, B, m = (np.asarray(v, float) for v in (W0, A, B, m))
+    sq = np.sum(W0 * W0, axis=1) + 2 * s * np.sum(B * (W0 @ A.T), axis=1) + s * np.sum(B * (B @ (A @ A.T)), axis=1)
+    C = np.sqrt(sq)
+    return C, m / C, (m - C) / C
+
+
 _V_no_s = lambda W0, A, B, s: np.asarray(W0, float) + np.asarray(B, float) @ np.asarray(A, float)
 _V_neg = lambda W0, A, B, s: np.asarray(W0, float) - s * (np.asarray(B, float) @ np.asarray(A, float))
 _V_s2 = lambda W0, A, B, s: np.asarray(W0, float) + s * s * (np.asarray(B, float) @ np.asarray(A, float))
@@ -371,6 +401,7 @@ MUTANTS = {
     "s_squared": _mutant(norm=_norm_using(_V_s2), forward=_forward_using(_V_s2)),
     "column_norm": _mutant(norm=_norm_using(_V, axis=0)),
     "gm1_flipped": _mutant(norm=_gm1_flipped),
+    "factored_gram_times_s": _mutant(norm_factored=_factored_gram_s),
     "forward_ignores_fixed_C": _mutant(forward=_forward_ignores_C),
     "dV_without_g": _mutant(backward=_backward_variant("no_g_in_dV")),
     "dm_over_C2": _mutant(backward=_backward_variant("dm_over_C2")),

@@ -48,10 +48,13 @@ def test_small_parity(name):
     dev = tl.to_device(inp)
     out = tl.run_gpu(dev, wl.s)
     ref = tl.run_oracle(inp)
-    tl.check_all(out, ref, wl.dtype, what=name)
-    # Intermediate saved for the backward: su = s x A^T.
+    tl.check_all(out, ref, inp, what=name)
+    # Intermediate saved for the backward: su = s x A^T, element by element.
     su_ref = wl.s * (inp["x"].astype(np.float64) @ inp["A"].astype(np.float64).T)
     tl.check_tensor("su", out["su"], su_ref, wl.dtype, what=name)
+    tl.check_elementwise("su", out["su"], su_ref, tl.element_bounds(inp, ref, out, wl.dtype)["su"], what=name)
+    if wl.m_lo is None:
+        tl.check_near_unity(out["y"], inp, ref, what=name)
 
 
 FULL = ["c2", "c3", "c4a", "c4b", "c5"]
@@ -65,7 +68,9 @@ def test_full_workload_parity(key):
     out = tl.run_gpu(dev, wl.s)
     del dev
     ref = tl.run_oracle(inp)
-    tl.check_all(out, ref, wl.dtype, what=wl.name)
+    tl.check_all(out, ref, inp, what=wl.name)
+    if wl.m_lo is None:  # c4a, c4b: g = 1 +- 1e-3, the adapted part of y must survive the rounding
+        tl.check_near_unity(out["y"], inp, ref, what=wl.name)
 
 
 def test_near_unity_gm1_resolution():

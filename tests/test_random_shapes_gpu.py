@@ -47,7 +47,7 @@ def test_random_shape_parity(shape):
     dev = tl.to_device(inp)
     out = tl.run_gpu(dev, wl.s)
     ref = tl.run_oracle(inp)
-    tl.check_all(out, ref, wl.dtype, what=f"{shape}")
+    tl.check_all(out, ref, inp, what=f"{shape}")
     W0, A, B, m, x, dy = (inp[k] for k in ("W0", "A", "B", "m", "x", "dy"))
     Wm = dw.dora_merge(dev["W0"], dev["A"], dev["B"], out["g"], wl.s)
     tl.check_tensor("W_merged", Wm, oracle.merge(W0, A, B, m, wl.s), "bf16", what=f"{shape}")

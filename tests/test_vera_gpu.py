@@ -47,22 +47,20 @@ def test_dvora_layer_step(key, ov):
     W0, A, x, dy, Bs_d = dev(inp["W0"]), dev(inp["A"]), dev(inp["x"]), dev(inp["dy"]), dev(Bs)
     m = dev(inp["m"], torch.float32)
     b_d, d_d = dev(b, torch.float32), dev(d, torch.float32)
-    Bp = dw.dora_vera_compose(Bs_d, b_d, d_d)
-    norm, g, gm1 = dw.dora_norm(W0, A, Bp, m, wl.s)
-    y, su, pre = dw.dora_forward(x, W0, A, Bp, gm1, wl.s)
-    dm, dA, dBp, dx = dw.dora_backward(dy, x, W0, A, Bp, norm, g, su, pre, wl.s)
-    db, dd = dw.dora_vera_grad(Bs_d, b_d, d_d, dBp)
+    Bp = dw.dora_vera_compose(Bs_d, b_d, d_d, out=tl.poisoned((wl.d_out, wl.r), dt))
+    out = tl.run_gpu({"W0": W0, "A": A, "B": Bp, "m": m, "x": x, "dy": dy}, wl.s)
+    dBp = out["dB"]
+    db, dd = dw.dora_vera_grad(Bs_d, b_d, d_d, dBp, db=tl.poisoned((wl.d_out,), torch.float32),
+                               dd=tl.poisoned((wl.r,), torch.float32))
 
     Bp_ref = oracle.vera_direction(Bs, b, d)
     # B' is rounded once from an fp32 product: within one rounding of the exact value.
     rel = np.abs(tl.host(Bp) - Bp_ref) / np.maximum(np.abs(Bp_ref), 1e-30)
     assert np.max(rel) <= (2.0 ** -8 if wl.dtype == "bf16" else 1e-6)
     # The rest against the oracle on the device's B' (the rounded values the layer really used).
-    Bp_used = tl.host(Bp)
-    ref_y = oracle.forward(inp["x"], inp["W0"], inp["A"], Bp_used, inp["m"], wl.s)
-    ref = oracle.backward(inp["dy"], inp["x"], inp["W0"], inp["A"], Bp_used, inp["m"], wl.s)
-    tl.check_tensor("y", y, ref_y, wl.dtype, what="dvora")
-    tl.check_tensor("dm", dm, ref["dm"], wl.dtype, what="dvora")
+    inp_used = dict(inp, B=tl.host(Bp))
+    ref = tl.run_oracle(inp_used)
+    tl.check_all(out, ref, inp_used, what="dvora")
     rdb, rdd = oracle.vera_gradients(ref["dB"], Bs, b, d)
     tl.check_tensor("db", db, rdb, wl.dtype, what="dvora")
     tl.check_tensor("dd", dd, rdd, wl.dtype, what="dvora")
