@@ -6,9 +6,10 @@ g - 1), dora_forward (LoRA down projection, base GEMM with the near-unity
 compose) and dora_backward (compose backward, du, dB, dA, dx), on the
 high-rank workload d_out = d_in = 8192, r = 384, s = 0.5, 4096 tokens, bf16.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload c1..c5]
+    python bench.py --table profiles/workloads.md     # every workload, one line each, plus a table
 
-Under torchrun (N > 1) every rank runs the step on its own 4096 tokens with
+Under torchrun (N > 1) every rank runs the step on its own tokens with
 replicated weights and the per-rank dm, dA, dB are summed with NCCL (weak
 scaling). Rank 0 prints one JSON line.
 
@@ -18,8 +19,8 @@ the events. Kernel durations come from the library's own event profiler on a
 second, profiled capture of the same calls. `e2e` runs the public Python API
 eagerly with every step's inputs copied from pinned host memory and its
 results copied back inside the timed region, the copies of neighbouring steps
-overlapping the compute on separate streams. `--impl reference` times the CPU float64 oracle
-on a bounded token sample of the same workload.
+overlapping the compute on separate streams. `--impl reference` times the CPU
+float64 oracle on whole steps of the same workload.
 """
 from __future__ import annotations
 
@@ -40,6 +41,7 @@ sys.path.insert(0, ROOT)
 METRIC = "DoRA layer fwd+bwd tokens/s and norm TFLOP/s at d_in=8192 r=384 bf16; % roofline"
 UNIT = "tokens/s"
 WORKLOAD_KEY = "c3"
+WORKLOAD_KEYS = ("c1", "c2", "c3", "c4a", "c4b", "c5")
 FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -54,14 +56,17 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=WORKLOAD_KEY, choices=["c2", "c3", "c4a", "c4b", "c5"],
-                    help="bf16 workload to time (default: the c3 layer the metric is quoted on)")
+    ap.add_argument("--workload", default=WORKLOAD_KEY, choices=list(WORKLOAD_KEYS),
+                    help="workload to time (default: the c3 layer the metric is quoted on)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--ref-tokens", type=int, default=256, help="tokens per reference-arm step")
-    ap.add_argument("--ref-rows", type=int, default=1024, help="output rows per reference-arm step")
+    ap.add_argument("--ref-budget-s", type=float, default=150.0,
+                    help="reference arm: wall-clock budget of the steps after the first; whole steps are timed "
+                         "while they fit, else a fixed share of the output rows with all tokens")
     ap.add_argument("--no-merge", action="store_true",
                     help="skip the inference, full-gradient, DVoRA and deployment-merge measurements")
+    ap.add_argument("--table", metavar="MD",
+                    help="time every workload (the layer step only) and write a markdown table to MD")
     return ap.parse_args(argv)
 
 
@@ -94,6 +99,52 @@ def kernel_work(name, wl):
         "merge_gemm": (2 * do * di * r + 3 * do * di, b * (2 * do * di + do * r + r * di) + 4 * do),
     }
     return table.get(name, (0, 0))
+
+
+def layer_roofline(wl, peaks):
+    """Roofline time of each call of the layer step at the measured burst peaks (bf16 workloads).
+
+    Each call is bound by the slower of its algorithmic flops at the dense
+    bf16 tensor peak and its algorithmic bytes at the HBM copy rate:
+      norm         2 d_out d_in r + 2 r^2 d_in + 2 d_out r^2 + 2 d_out d_in + 2 d_out r flops;
+                   W0, A, B once + C, g, g - 1 (fp32)
+      forward      2 T d_in (d_out + r) + 2 T r d_out flops; x, W0, A, B, s u (written and read), y and pre
+      compose bwd  dy, pre in and dz out (HBM only)
+      bwd GEMMs    2 T d_out d_in + 4 T d_out r + 4 T r d_in flops; dz, W0, x (twice), dx, du (written and read)
+    Returns ({call: seconds}, total seconds), or (None, None) for fp32 layers.
+    """
+    if wl.dtype != "bf16":
+        return None, None
+    T, di, do, r = wl.T, wl.d_in, wl.d_out, wl.r
+    P, BW = peaks["bf16_tflops"] * 1e12, peaks["hbm_gbs"] * 1e9
+    b = 2
+    work = {
+        "norm": (2 * do * di * r + 2 * r * r * di + 2 * do * r * r + 2 * do * di + 2 * do * r,
+                 b * (do * di + r * di + do * r) + 12 * do),
+        "forward": (2 * T * di * (do + r) + 2 * T * r * do,
+                    b * (T * di + do * di + r * di + do * r + 2 * T * r + 2 * T * do)),
+        "compose_bwd": (0, b * 3 * T * do + 4 * do),
+        "bwd_gemms": (2 * T * do * di + 4 * T * do * r + 4 * T * r * di,
+                      b * (T * do + do * di + 2 * T * di + T * di + 2 * T * r + r * di + do * r)),
+    }
+    t = {k: max(f / P, by / BW) for k, (f, by) in work.items()}
+    return t, sum(t.values())
+
+
+def norm_flops(wl):
+    T, di, do, r = wl.T, wl.d_in, wl.d_out, wl.r
+    return 2 * do * di * r + 2 * r * r * di + 2 * do * r * r + 2 * do * di + 2 * do * r
+
+
+def sig(v, n=4):
+    """Round floats (recursively) to n significant digits, to keep the JSON line short."""
+    if isinstance(v, float):
+        return float(f"{v:.{n}g}") if v == v and abs(v) != float("inf") else v
+    if isinstance(v, dict):
+        return {k: sig(x, n) for k, x in v.items()}
+    if isinstance(v, (list, tuple)):
+        return [sig(x, n) for x in v]
+    return v
 
 
 # Source files that define each kernel: DRAM traffic recorded by ncu stays
@@ -228,12 +279,24 @@ def blas_threads():
         return os.cpu_count()
 
 
-def oracle_step(inp, T, rows=None):
-    """Oracle norm + forward + backward on the first T tokens (and, if given,
-    the first `rows` output features: a smaller layer with the same d_in and r)."""
+def oracle_inputs(wl):
+    """Seeded inputs; near-unity workloads get m = C (1 + delta) from the oracle's own C."""
+    import numpy as np
+    import oracle
+    from dora_inputs import make_inputs, near_unity_magnitude
+    inp = make_inputs(wl)
+    if inp["m"] is None:
+        C, _, _ = oracle.norm(inp["W0"], inp["A"], inp["B"], np.ones(wl.d_out), inp["s"])
+        inp["m"] = near_unity_magnitude(C, inp["delta"])
+    return inp
+
+
+def oracle_step(inp, rows=None):
+    """Oracle norm + forward + backward on all tokens (and, if given, the first
+    `rows` output features: a smaller layer with the same d_in, r and T)."""
     import oracle
     W0, A, B, m, s = (inp[k] for k in ("W0", "A", "B", "m", "s"))
-    x, dy = inp["x"][:T], inp["dy"][:T]
+    x, dy = inp["x"], inp["dy"]
     if rows is not None:
         W0, B, m, dy = W0[:rows], B[:rows], m[:rows], dy[:, :rows]
     oracle.norm(W0, A, B, m, s)
@@ -241,77 +304,117 @@ def oracle_step(inp, T, rows=None):
     oracle.backward(dy, x, W0, A, B, m, s)
 
 
-def time_oracle(inp, T, min_seconds=10.0, max_steps=3):
+def time_oracle(inp, min_seconds=10.0, max_steps=3):
     steps, t0 = 0, time.perf_counter()
     while True:
-        oracle_step(inp, T)
+        oracle_step(inp)
         steps += 1
         el = time.perf_counter() - t0
         if el >= min_seconds or steps >= max_steps:
             return steps, el
 
 
+def time_oracle_norms(inp, wl, reps=2):
+    """The norm alone on the CPU: the dense definition and the factored form (fp64)."""
+    import oracle
+    args = tuple(inp[k] for k in ("W0", "A", "B", "m", "s"))
+    out = {}
+    for name, fn in (("dense", oracle.norm), ("factored", oracle.norm_factored)):
+        fn(*args)
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            fn(*args)
+        sec = (time.perf_counter() - t0) / reps
+        out[name] = {"ms": 1e3 * sec, "tflops": norm_flops(wl) / sec / 1e12}
+    return out
+
+
 # ---------------------------------------------------------------- reference arm
 
 def run_reference(args, wl, cfg):
-    from dora_inputs import make_inputs
+    """The oracle (the reference arm: CPU float64, dense W0 + s B A) on whole steps.
+
+    The first warm-up step runs the whole layer and measures it. The remaining
+    warm-up and the K timed steps run the whole layer too when they fit the
+    wall-clock budget; otherwise each runs all T tokens on the first `rows`
+    output features (a multiple of 64), and the rate is scaled by d_out / rows,
+    which is exact for this step: every term of norm, forward and backward is
+    linear in d_out at fixed T (the rows are independent until dA sums them).
+    """
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
-        return 0
-    inp = make_inputs(wl)
-    T = min(args.ref_tokens, wl.T)
-    rows = min(args.ref_rows, wl.d_out)
-    for _ in range(args.warmup):
-        oracle_step(inp, T, rows)
+        return None
+    inp = oracle_inputs(wl)
+    t0 = time.perf_counter()
+    oracle_step(inp)
+    t_full = time.perf_counter() - t0
+    rest = max(args.warmup - 1, 0) + args.steps
+    rows = wl.d_out
+    if rest * t_full > args.ref_budget_s:
+        rows = max(64, int(wl.d_out * args.ref_budget_s / (rest * t_full)) // 64 * 64)
+        rows = min(rows, wl.d_out)
+    for _ in range(max(args.warmup - 1, 0)):
+        oracle_step(inp, rows)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(inp, T, rows)
+        oracle_step(inp, rows)
     el = time.perf_counter() - t0
-    # Every term of the layer step is linear in d_out, so a step of the full
-    # layer costs d_out / rows sample steps.
     full_step_s = (el / args.steps) * (wl.d_out / rows)
-    value = T / full_step_s
+    value = wl.T / full_step_s
+    if rows == wl.d_out:
+        sample = (f"{args.steps} whole steps of the {wl.name} layer ({wl.T} tokens, {wl.d_out} output rows; "
+                  f"norm + forward + backward in float64 NumPy, dense W0 + s*B*A), measured")
+    else:
+        sample = (f"{args.steps} steps of all {wl.T} tokens on {rows} of {wl.d_out} output rows of the {wl.name} "
+                  f"layer (float64 NumPy, dense W0 + s*B*A); rate scaled by d_out / rows (the step is linear in "
+                  f"d_out); one whole step measured {t_full:.2f} s")
     cores = blas_threads()
-    sample = (f"{T} of {wl.T} tokens and {rows} of {wl.d_out} output rows per step of the {wl.name} layer "
-              f"(norm + forward + backward in float64 NumPy, dense W0 + s*B*A), {args.steps} steps; "
-              f"rate scaled by rows / d_out to the full layer")
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * full_step_s, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
-            "impl": "reference",
+            "impl": "reference", "whole_step_s": t_full,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-    print(json.dumps(line), flush=True)
-    return 0
+    return sig(line, 6)
 
 
 # ---------------------------------------------------------------- our arm
 
-def run_ours(args, wl, cfg):
+def graph_time_ms(torch, fn, flush, warmup, calls):
+    """Median device time of one CUDA-graph replay of fn (L2 flushed before each)."""
+    fn()
+    gph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gph):
+        fn()
+    ev = []
+    for i in range(max(3, warmup) + calls):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        gph.replay()
+        e1.record()
+        if i >= max(3, warmup):
+            ev.append((e0, e1))
+    torch.cuda.synchronize()
+    del gph
+    return statistics.median(a.elapsed_time(b) for a, b in ev), len(ev)
+
+
+def run_ours(args, wl, cfg, dist=None, extras=True):
     import numpy as np
     import torch
     import dora_weight_decomposed_b200 as dw
-    from dora_weight_decomposed_b200 import build as dbuild
     from dora_weight_decomposed_b200.dp import allreduce_gradients
     from dora_inputs import make_inputs
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus:
-        log(f"note: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE")
-    torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
-    dbuild.build()
-    dw.load_library()
 
     inp = make_inputs(wl, token_seed=rank)
-    bf = torch.bfloat16
-    td = {k: torch.from_numpy(inp[k]).to(dev).to(bf).contiguous() for k in ("W0", "A", "B", "x", "dy")}
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    td = {k: torch.from_numpy(inp[k]).to(dev).to(dt).contiguous() for k in ("W0", "A", "B", "x", "dy")}
     W0, A, B, x, dy, s = td["W0"], td["A"], td["B"], td["x"], td["dy"], wl.s
     if inp["m"] is not None:
         m = torch.from_numpy(inp["m"]).to(dev)
@@ -325,14 +428,14 @@ def run_ours(args, wl, cfg):
     T, di, do, r = wl.T, wl.d_in, wl.d_out, wl.r
     f32 = dict(device=dev, dtype=torch.float32)
     C, g, gm1 = torch.empty(do, **f32), torch.empty(do, **f32), torch.empty(do, **f32)
-    y = torch.empty(T, do, device=dev, dtype=bf)
-    su = torch.empty(T, r, device=dev, dtype=bf)
-    pre = torch.empty(T, do, device=dev, dtype=bf)
+    y = torch.empty(T, do, device=dev, dtype=dt)
+    su = torch.empty(T, r, device=dev, dtype=dt)
+    pre = torch.empty(T, do, device=dev, dtype=dt)
     dm = torch.empty(do, **f32)
-    dA = torch.empty(r, di, device=dev, dtype=bf)
-    dB = torch.empty(do, r, device=dev, dtype=bf)
-    dx = torch.empty(T, di, device=dev, dtype=bf)
-    ws = [torch.empty(max(dw.dora_workspace_size(do, di, r, bf, s, T, op), 256), dtype=torch.uint8, device=dev)
+    dA = torch.empty(r, di, device=dev, dtype=dt)
+    dB = torch.empty(do, r, device=dev, dtype=dt)
+    dx = torch.empty(T, di, device=dev, dtype=dt)
+    ws = [torch.empty(max(dw.dora_workspace_size(do, di, r, dt, s, T, op), 256), dtype=torch.uint8, device=dev)
           for op in (dw.DORA_OP_NORM, dw.DORA_OP_FORWARD, dw.DORA_OP_BACKWARD)]
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
@@ -369,16 +472,13 @@ def run_ours(args, wl, cfg):
     prof = capture(True)
     launches_per_step = dw.dora_profile_count()
 
-    def replay(graphs):
-        for gph in graphs:
-            gph.replay()
-        if dist is not None:
-            allreduce_gradients(dm, dA, dB)
-
     # ---- warm-up
     for _ in range(args.warmup):
         flush.zero_()
-        replay(plain)
+        for gph in plain:
+            gph.replay()
+        if dist is not None:
+            allreduce_gradients(dm, dA, dB)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
@@ -418,6 +518,7 @@ def run_ours(args, wl, cfg):
         total_ms = float(t.item())
     ms_per_step = total_ms / args.steps
     value = world * T * args.steps / (total_ms / 1e3)
+    del plain
 
     # ---- per-kernel durations from the profiled capture
     nprof = min(args.steps, 50)
@@ -429,33 +530,82 @@ def run_ours(args, wl, cfg):
         torch.cuda.synchronize()
         for name, ms in dw.dora_profile_read():
             per.setdefault(name, []).append(ms)
+    del prof
+    peaks, peak_src = load_peaks()
+    P_burst, P_sus, BW = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"], peaks["hbm_gbs"]
     kernels = {}
     for name, v in per.items():
         launches = len(v) / nprof
         avg = sum(v) / len(v)
-        fl, by = kernel_work(name, wl)
-        kernels[name] = {"ms": avg, "launches_per_step": launches, "share": 0.0,
-                         "tflops": (fl / (avg * 1e-3) / 1e12) if fl else None,
-                         "gbs": (by / (avg * 1e-3) / 1e9) if by else None}
-    tot = sum(k["ms"] * k["launches_per_step"] for k in kernels.values()) or 1.0
+        fl, by = kernel_work(name, wl) if wl.dtype == "bf16" else (0, 0)
+        tf = fl / (avg * 1e-3) / 1e12 if fl else None
+        gb = by / (avg * 1e-3) / 1e9 if by else None
+        # Fraction of the kernel's own bound (the slower of its tensor and HBM times at the burst peaks).
+        frac = None
+        if fl or by:
+            frac = max((tf or 0.0) / P_burst, (gb or 0.0) / BW) if name != "compose_bwd" else gb / BW
+        kernels[name] = {"us": 1e3 * avg, "n": launches, "tflops": tf, "gbs": gb, "frac": frac}
+    tot = sum(k["us"] * k["n"] for k in kernels.values()) or 1.0
     for k in kernels.values():
-        k["share"] = k["ms"] * k["launches_per_step"] / tot
-    dom = max(kernels, key=lambda n: kernels[n]["ms"] * kernels[n]["launches_per_step"])
-    peaks, peak_src = load_peaks()
+        k["share"] = k["us"] * k["n"] / tot
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic", "config": cfg,
+            "gpu_launches": int(launches_per_step * args.steps), "clocks": clocks.summary(),
+            "step_ms_min": min(step_ms), "step_ms_median": statistics.median(step_ms),
+            "call_us": {k: 1e3 * v for k, v in phase_ms.items()}}
+    t_roof, t_roof_total = layer_roofline(wl, peaks)
+    if t_roof is not None:
+        line["layer_roofline"] = {"us": 1e6 * t_roof_total, "tokens_per_s": world * T / t_roof_total,
+                                  "frac": 1e3 * t_roof_total / ms_per_step,
+                                  "call_us": {k: 1e6 * v for k, v in t_roof.items()},
+                                  "peaks": "measured burst bf16 and HBM copy"}
+    if wl.dtype != "bf16":
+        line["kernels"] = {n: [k["us"], k["n"]] for n, k in kernels.items()}
+        line["roofline"] = None
+        line["note"] = "fp32 layer on the SIMT path: launch-bound at this size, no roofline"
+        return line
+
+    # Dominant kernel: its own roofline against the burst peak (it is timed per launch inside a short,
+    # L2-flushed step); the sustained-peak fraction is reported beside it.
+    dom = max(kernels, key=lambda n: kernels[n]["us"] * kernels[n]["n"])
     fl, by = kernel_work(dom, wl)
-    d_ms = kernels[dom]["ms"]
+    d_s = kernels[dom]["us"] * 1e-6
     if dom == "compose_bwd":
-        roof = {"bound": "hbm", "achieved": by / (d_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+        roof = {"bound": "hbm", "achieved": by / d_s / 1e9, "peak": BW, "unit": "GB/s"}
+        roof["peak_source"] = f"{peak_src} (hbm_gbs)"
     else:
-        roof = {"bound": "tensor", "achieved": fl / (d_ms * 1e-3) / 1e12, "peak": peaks["bf16_tflops_sustained"],
-                "unit": "TFLOP/s"}
+        roof = {"bound": "tensor", "achieved": fl / d_s / 1e12, "peak": P_burst, "unit": "TFLOP/s"}
+        roof["peak_source"] = f"{peak_src} (bf16_tflops, burst)"
+        roof["frac_of_sustained"] = roof["achieved"] / P_sus
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["kernel"] = dom
-    roof["peak_source"] = f"{peak_src} ({'bf16_tflops_sustained' if roof['unit'] == 'TFLOP/s' else 'hbm_gbs'})"
-    tr = recorded_traffic(dom)
-    roof["traffic"] = tr
+    roof["traffic"] = recorded_traffic(dom)
     roof["algorithmic_per_launch"] = fl if roof["unit"] == "TFLOP/s" else by
-    norm_flops = (2 * do * di * r + 2 * r * r * di + 2 * do * r * r + 2 * do * di + 2 * do * r)
+    roof["kernel"] = dom
+
+    nf = norm_flops(wl)
+    norm_call_tflops = nf / (phase_ms["norm"] * 1e-3) / 1e12
+    nk = kernels.get("norm_gemm")
+    norm_roof = {"bound": "tensor", "achieved": norm_call_tflops, "peak": P_burst, "unit": "TFLOP/s",
+                 "frac": norm_call_tflops / P_burst, "call_us": 1e3 * phase_ms["norm"],
+                 "flops": nf, "peak_source": f"{peak_src} (bf16_tflops, burst)"}
+    if nk is not None:
+        norm_roof["norm_gemm_us"] = nk["us"]
+        norm_roof["norm_gemm_tflops"] = nk["tflops"]
+        norm_roof["norm_gemm_frac"] = nk["frac"]
+    cb = kernels.get("compose_bwd")
+    cb_roof = None
+    if cb is not None:
+        cb_roof = {"bound": "hbm", "achieved": cb["gbs"], "peak": BW, "unit": "GB/s", "frac": cb["gbs"] / BW,
+                   "us": cb["us"], "bytes": kernel_work("compose_bwd", wl)[1],
+                   "peak_source": f"{peak_src} (hbm_gbs)"}
+    line["kernels"] = {n: [k["us"], k["n"], k["frac"]] for n, k in kernels.items()}
+    line["kernels_fields"] = ["us per launch", "launches per step", "fraction of the kernel's bound (burst peaks)"]
+    if not extras:
+        line.update({"norm_tflops": norm_call_tflops, "norm_roofline": norm_roof, "compose_bwd_roofline": cb_roof,
+                     "roofline": roof})
+        return line
 
     # ---- end to end through the public API with host buffers
     # Every step copies its inputs (x, dy, and the trained A, B, m) from pinned
@@ -531,150 +681,107 @@ def run_ours(args, wl, cfg):
                "l2": "not flushed: every step's inputs and W0 exceed L2"}
         del sets
 
-    # ---- cached-norm inference: forward only, norm reused, nothing saved for a backward
-    infer = None
+    # ---- the next rows on the same layer, each one CUDA graph per call, L2 flushed before each:
+    # cached-norm inference (forward only, nothing saved), the full gradient (appendix A eq. A.1),
+    # DVoRA's two passes and the deployment merge.
+    side = {}
     if rank == 0 and not args.no_merge:
-        wsi = torch.empty(max(dw.dora_workspace_size(do, di, r, bf, s, T, dw.DORA_OP_FORWARD), 256),
+        wsi = torch.empty(max(dw.dora_workspace_size(do, di, r, dt, s, T, dw.DORA_OP_FORWARD), 256),
                           dtype=torch.uint8, device=dev)
-        call_inf = lambda: dw.dora_forward(x, W0, A, B, gm1, s, y=y, save_for_backward=False, ws=wsi)
-        call_inf()
-        gi = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gi):
-            call_inf()
-        iev = []
-        for i in range(max(3, args.warmup) + 20):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            gi.replay()
-            e1.record()
-            if i >= max(3, args.warmup):
-                iev.append((e0, e1))
-        torch.cuda.synchronize()
-        i_ms = statistics.median(a.elapsed_time(b_) for a, b_ in iev)
+        i_ms, n = graph_time_ms(torch, lambda: dw.dora_forward(x, W0, A, B, gm1, s, y=y, save_for_backward=False,
+                                                               ws=wsi), flush, args.warmup, 20)
         fl = 2 * T * do * (di + r) + 2 * T * di * r
-        infer = {"value": T / (i_ms * 1e-3), "unit": UNIT, "ms_per_batch": i_ms, "tflops": fl / (i_ms * 1e-3) / 1e12,
-                 "calls": len(iev), "api": "dora_forward(save_for_backward=False) with the norm of a prior dora_norm",
-                 "l2": "flushed before every call"}
-        del gi, wsi
-
-    # ---- the backward without the detach of the norm (appendix A eq. A.1), same layer and batch
-    full_bwd = None
-    if rank == 0 and not args.no_merge:
-        wsf = torch.empty(max(dw.dora_workspace_size(do, di, r, bf, s, T, dw.DORA_OP_BACKWARD_FULL), 256),
+        side["inference"] = {"tokens_per_s": T / (i_ms * 1e-3), "us": 1e3 * i_ms,
+                             "tflops": fl / (i_ms * 1e-3) / 1e12}
+        del wsi
+        wsf = torch.empty(max(dw.dora_workspace_size(do, di, r, dt, s, T, dw.DORA_OP_BACKWARD_FULL), 256),
                           dtype=torch.uint8, device=dev)
-        call_full = lambda: dw.dora_backward_full(dy, x, W0, A, B, C, g, su, pre, s, dm=dm, dA=dA, dB=dB, dx=dx,
-                                                  ws=wsf)
-        call_full()
-        gf = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gf):
-            call_full()
-        fev = []
-        for i in range(max(3, args.warmup) + 20):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            gf.replay()
-            e1.record()
-            if i >= max(3, args.warmup):
-                fev.append((e0, e1))
-        torch.cuda.synchronize()
-        f_ms = statistics.median(a.elapsed_time(b_) for a, b_ in fev)
-        full_bwd = {"ms": f_ms, "detached_ms": phase_ms["backward"], "calls": len(fev),
-                    "api": "dora_backward_full", "l2": "flushed before every call"}
-        del gf, wsf
-
-    # ---- DVoRA's extra calls on the same layer: form B' = diag(b) B diag(d), and db, dd from dB'
-    vera = None
-    if rank == 0 and not args.no_merge:
+        f_ms, _ = graph_time_ms(torch, lambda: dw.dora_backward_full(dy, x, W0, A, B, C, g, su, pre, s, dm=dm, dA=dA,
+                                                                     dB=dB, dx=dx, ws=wsf), flush, args.warmup, 20)
+        side["backward_full"] = {"us": 1e3 * f_ms, "detached_us": 1e3 * phase_ms["backward"]}
+        del wsf
         bv = torch.linspace(0.5, 1.5, do, device=dev)
         dv = torch.linspace(-1.0, 1.0, r, device=dev)
         Bp = torch.empty_like(B)
-        wsv = torch.empty(max(dw.dora_workspace_size(do, 8, r, bf, 1.0, 0, dw.DORA_OP_VERA_GRAD), 256),
+        wsv = torch.empty(max(dw.dora_workspace_size(do, 8, r, dt, 1.0, 0, dw.DORA_OP_VERA_GRAD), 256),
                           dtype=torch.uint8, device=dev)
-        timings = {}
+        vb = {"compose": 2 * (2 * do * r) + 4 * (do + r), "grad": 2 * (2 * do * r) + 8 * (do + r)}
         for name, fn in (("compose", lambda: dw.dora_vera_compose(B, bv, dv, out=Bp)),
                          ("grad", lambda: dw.dora_vera_grad(B, bv, dv, dB, ws=wsv))):
-            fn()
-            gv = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gv):
-                fn()
-            vev = []
-            for i in range(max(3, args.warmup) + 20):
-                flush.zero_()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-                gv.replay()
-                e1.record()
-                if i >= max(3, args.warmup):
-                    vev.append((e0, e1))
-            torch.cuda.synchronize()
-            timings[name] = statistics.median(a.elapsed_time(b_) for a, b_ in vev)
-            del gv
-        vb = {"compose": 2 * (2 * do * r) + 4 * (do + r), "grad": 2 * (2 * do * r) + 8 * (do + r)}
-        vera = {k: {"us": timings[k] * 1e3, "gbs": vb[k] / (timings[k] * 1e-3) / 1e9} for k in timings}
-        vera["api"] = "dora_vera_compose, dora_vera_grad (one CUDA graph per call, L2 flushed)"
+            v_ms, _ = graph_time_ms(torch, fn, flush, args.warmup, 20)
+            side[f"dvora_{name}"] = {"us": 1e3 * v_ms, "gbs": vb[name] / (v_ms * 1e-3) / 1e9}
         del Bp, wsv
-
-    # ---- deployment merge W' = diag(g) (W0 + s B A) on the same layer (not part of the step)
-    merge = None
-    if rank == 0 and not args.no_merge:
         Wm = torch.empty_like(W0)
-        call_merge = lambda: dw.dora_merge(W0, A, B, g, s, out=Wm)
-        for _ in range(3):
-            call_merge()
-        gm = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gm):
-            call_merge()
-        mev = []
-        for _ in range(20):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            gm.replay()
-            e1.record()
-            mev.append((e0, e1))
-        torch.cuda.synchronize()
-        del gm
-        m_ms = statistics.median(a.elapsed_time(b_) for a, b_ in mev)
+        m_ms, _ = graph_time_ms(torch, lambda: dw.dora_merge(W0, A, B, g, s, out=Wm), flush, 3, 20)
+        del Wm
         fl, by = kernel_work("merge_gemm", wl)
         gbs, tfl = by / (m_ms * 1e-3) / 1e9, fl / (m_ms * 1e-3) / 1e12
         # Bound: the larger of HBM time and tensor time at the measured burst peaks.
-        hbm_bound = by / peaks["hbm_gbs"] >= fl / (peaks["bf16_tflops"] * 1e3)
-        mroof = ({"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s"} if hbm_bound else
-                 {"bound": "tensor", "achieved": tfl, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"})
+        hbm_bound = by / BW >= fl / (P_burst * 1e3)
+        mroof = ({"bound": "hbm", "achieved": gbs, "peak": BW, "unit": "GB/s"} if hbm_bound else
+                 {"bound": "tensor", "achieved": tfl, "peak": P_burst, "unit": "TFLOP/s"})
         mroof["frac"] = mroof["achieved"] / mroof["peak"]
-        mroof["peak_source"] = f"{peak_src} ({'hbm_gbs' if hbm_bound else 'bf16_tflops'}, burst)"
         mroof["traffic"] = recorded_traffic("merge_gemm")
-        merge = {"us": m_ms * 1e3, "gbs": gbs, "tflops": tfl, "calls": len(mev), "roofline": mroof,
-                 "l2": "flushed before every call", "api": "dora_merge (one CUDA graph per call)"}
-        del Wm
+        side["merge"] = {"us": 1e3 * m_ms, "tflops": tfl, "roofline": mroof}
+        side["timing"] = "one CUDA graph per call, L2 flushed before each, median of 20"
 
     status = dw.dora_device_status()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        steps, el = time_oracle(inp, T)
+        oinp = inp if inp["m"] is not None else oracle_inputs(wl)
+        steps, el = time_oracle(oinp)
+        norms = time_oracle_norms(oinp, wl)
         cpu = {"value": T * steps / el, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                "sample": f"{steps} full step(s) of {T} tokens on the {wl.name} layer in float64 NumPy "
-                         f"(dense W0 + s*B*A; norm + forward + backward), {el:.1f} s"}
+                         f"(dense W0 + s*B*A; norm + forward + backward), {el:.1f} s",
+               "norm_dense": norms["dense"], "norm_factored": norms["factored"]}
 
-    if dist is not None:
-        del plain, prof
-        dist.destroy_process_group()
-    if rank != 0:
-        return 0
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
-            "norm_tflops": norm_flops / (phase_ms["norm"] * 1e-3) / 1e12, "phase_ms": phase_ms,
-            "roofline": roof, "kernels": kernels, "inference": infer, "backward_full": full_bwd, "merge": merge,
-            "dvora": vera,
-            "gpu_launches": int(launches_per_step * args.steps),
-            "clocks": clocks.summary(), "e2e": e2e, "cpu_baseline": cpu, "device_status": status,
-            "step_ms_min": min(step_ms), "step_ms_median": statistics.median(step_ms)}
-    print(json.dumps(line), flush=True)
+    line.update({"next_rows": side, "device_status": status, "e2e": e2e, "cpu_baseline": cpu,
+                 "norm_tflops": norm_call_tflops, "norm_roofline": norm_roof, "compose_bwd_roofline": cb_roof,
+                 "roofline": roof})
+    return line
+
+
+def _table(args):
+    """Every workload in turn (the layer step only): one JSON line each and a markdown table."""
+    import torch
+    from dora_inputs import workload
+    rows = []
+    for key in WORKLOAD_KEYS:
+        wl = workload(key)
+        cfg = workload_config(wl, 1)
+        line = run_ours(args, wl, cfg, extras=False)
+        print(json.dumps(sig(line)), flush=True)
+        rows.append((key, wl, line))
+        torch.cuda.empty_cache()
+    out = ["| workload | dtype | tokens/s | µs per step | norm / forward / backward µs | layer roofline µs "
+           "(tokens/s) | fraction of roofline | norm TFLOP/s | launches per step |",
+           "|---|---|---|---|---|---|---|---|---|"]
+    for key, wl, l in rows:
+        c = l["call_us"]
+        lr = l.get("layer_roofline")
+        roof = f"{lr['us']:.1f} ({lr['tokens_per_s'] / 1e6:.2f} M)" if lr else "— (launch-bound)"
+        frac = f"{lr['frac']:.2f}" if lr else "—"
+        ntf = f"{l['norm_tflops']:.0f}" if "norm_tflops" in l else "—"
+        out.append(f"| {key} {wl.d_out}×{wl.d_in} r={wl.r} T={wl.T} | {wl.dtype} | {l['value'] / 1e6:.3f} M | "
+                   f"{1e3 * l['ms_per_step']:.1f} | {c['norm']:.1f} / {c['forward']:.1f} / {c['backward']:.1f} | "
+                   f"{roof} | {frac} | {ntf} | {l['gpu_launches'] // max(args.steps, 1)} |")
+    clk = rows[-1][2]["clocks"]
+    out.append("")
+    out.append(f"Last workload's clocks: median {clk.get('sm_mhz')} MHz of {clk.get('sm_max_mhz')}, "
+               f"reasons {clk.get('reasons')}.")
+    with open(args.table, "w") as f:
+        f.write("\n".join(out) + "\n")
+    log("\n".join(out))
     return 0
+
+
+def workload_config(wl, world):
+    return {"workload": wl.name, "d_out": wl.d_out, "d_in": wl.d_in, "r": wl.r, "s": wl.s,
+            "tokens_per_gpu": wl.T, "global_tokens": wl.T * world, "parallelism": f"dp{world}",
+            "l2": "flushed before every timed step (256 MB write)",
+            "timing": "CUDA graphs per call, CUDA events per step, max over ranks"}
 
 
 def main(argv=None):
@@ -682,15 +789,38 @@ def main(argv=None):
     from dora_inputs import workload
     wl = workload(args.workload)
     world = int(os.environ.get("WORLD_SIZE", "1"))
-    cfg = {"workload": wl.name, "d_out": wl.d_out, "d_in": wl.d_in, "r": wl.r, "s": wl.s,
-           "tokens_per_gpu": wl.T, "global_tokens": wl.T * world, "parallelism": f"dp{world}",
-           "l2": "flushed before every timed step (256 MB write)",
-           "timing": "CUDA graphs per call, CUDA events per step, max over ranks"}
+    cfg = workload_config(wl, world)
     if args.impl == "reference":
         cfg["timing"] = "wall clock over the CPU oracle steps"
         cfg["l2"] = "not applicable (host CPU)"
-        return run_reference(args, wl, cfg)
-    return run_ours(args, wl, cfg)
+        line = run_reference(args, wl, cfg)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+    import torch
+    from dora_weight_decomposed_b200 import build as dbuild
+    import dora_weight_decomposed_b200 as dw
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        log(f"note: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE")
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dbuild.build()
+    dw.load_library()
+    if args.table:
+        return _table(args)
+    line = run_ours(args, wl, cfg, dist=dist)
+    if dist is not None:
+        dist.destroy_process_group()
+    if int(os.environ.get("RANK", "0")) == 0:
+        # The per-kernel table in full on stderr; the JSON line (rounded) on stdout.
+        log(json.dumps({"kernels_detail": line.get("kernels")}))
+        print(json.dumps(sig(line)), flush=True)
+    return 0
 
 
 if __name__ == "__main__":

@@ -18,7 +18,22 @@ def token_shard(T_total: int, rank: int, world: int) -> tuple[int, int]:
 
 
 def allreduce_gradients(dm, dA, dB, group=None) -> None:
-    """Sum dm, dA and dB over the data-parallel group, in place."""
+    """Sum dm, dA and dB over the data-parallel group, in place, in one float32 all-reduce.
+
+    bf16 gradients are widened to float32 before the sum and rounded once after
+    it: a bf16 all-reduce would round at every hop of the ring, so its error
+    would grow with the number of ranks. dm is float32 already. One flat buffer
+    carries all three, so the exchange is a single collective (float64 when
+    any of them is float64).
+    """
+    import torch
     import torch.distributed as dist
-    for t in (dm, dA, dB):
-        dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+    ts = (dm, dA, dB)
+    acc = torch.float64 if any(t.dtype == torch.float64 for t in ts) else torch.float32
+    flat = torch.cat([t.reshape(-1).to(acc) for t in ts])
+    dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
+    off = 0
+    for t in ts:
+        n = t.numel()
+        t.copy_(flat[off:off + n].view(t.shape))
+        off += n

@@ -1,8 +1,10 @@
-"""Data-parallel host logic on CPU: two gloo ranks, each with its own token
+"""Data-parallel host logic on CPU: gloo ranks, each with its own token
 shard, sum their per-rank gradients with dora_weight_decomposed_b200.dp and
 must get the gradients of the whole batch. The per-rank gradients come from
 the CPU oracle (no GPU here); on GPUs bench.py runs the same exchange over
-NCCL after the library's backward.
+NCCL after the library's backward. With four ranks the per-rank gradients are
+rounded to bf16 as the library stores them: the sum must then be rounded only
+once (float32 all-reduce), not once per hop as a bf16 all-reduce would.
 """
 import os
 import socket
@@ -79,3 +81,66 @@ def test_token_shard_covers_batch():
             assert max(sizes) - min(sizes) <= 1
     with pytest.raises(ValueError):
         token_shard(4, 2, 2)
+
+
+def _bf16_rank_main(rank, world, port, q):
+    import sys
+    sys.path.insert(0, ROOT)
+    import oracle
+    from dora_inputs import make_inputs, round_to_bf16, workload
+    from dora_weight_decomposed_b200.dp import allreduce_gradients, token_shard
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        T = 64
+        wl = workload("c2", d_out=48, d_in=40, r=8, T=T)
+        inp = make_inputs(wl)
+        W0, A, B, m, s = (inp[k] for k in ("W0", "A", "B", "m", "s"))
+        per_rank = []
+        for q_rank in range(world):  # every rank's bf16 gradients, to form the exact sum here
+            a, b = token_shard(T, q_rank, world)
+            gr = oracle.backward(inp["dy"][a:b], inp["x"][a:b], W0, A, B, m, s)
+            per_rank.append({k: round_to_bf16(gr[k]).astype(np.float64) for k in ("dA", "dB")} |
+                            {"dm": gr["dm"].astype(np.float32).astype(np.float64)})
+        mine = per_rank[rank]
+        dm = torch.from_numpy(mine["dm"].astype(np.float32))
+        dA = torch.from_numpy(mine["dA"].astype(np.float32)).to(torch.bfloat16)
+        dB = torch.from_numpy(mine["dB"].astype(np.float32)).to(torch.bfloat16)
+        allreduce_gradients(dm, dA, dB)
+        res = {}
+        for k, t in (("dm", dm), ("dA", dA), ("dB", dB)):
+            exact = sum(p[k] for p in per_rank)
+            mag = sum(np.abs(p[k]) for p in per_rank)
+            u = 2.0 ** -8 if k != "dm" else 2.0 ** -24
+            got = t.float().numpy().astype(np.float64)
+            # one rounding to the storage type + float32 summation of `world` terms
+            bound = u * np.abs(exact) + world * 2.0 ** -24 * mag
+            res[k] = float(np.max(np.abs(got - exact) / np.maximum(bound, 1e-300)))
+            # what a bf16 sum in ring order would give: a rounding after every addition
+            if k != "dm":
+                acc = per_rank[0][k]
+                for p in per_rank[1:]:
+                    acc = round_to_bf16(acc + p[k]).astype(np.float64)
+                res[k + "_bf16_ring_worst"] = float(np.max(np.abs(acc - exact) / np.maximum(bound, 1e-300)))
+        q.put((rank, res))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_four_rank_bf16_gradients_are_rounded_once():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    world = 4
+    procs = [ctx.Process(target=_bf16_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=180) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, res in results:
+        for k in ("dm", "dA", "dB"):
+            assert res[k] <= 1.0, f"rank {rank} {k}: error {res[k]:.2f} x the one-rounding bound"
+        # The test can tell the two apart: rounding at every hop leaves the bound somewhere.
+        assert max(res["dA_bf16_ring_worst"], res["dB_bf16_ring_worst"]) > 1.0
