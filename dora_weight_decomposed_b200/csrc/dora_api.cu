@@ -105,6 +105,36 @@ static NarrowChoice choose_narrow_1cta(int64_t M, int64_t N, int64_t K, bool b_m
   return best;
 }
 
+// Tile width and pairs per cluster (K splits reduced in the cluster) of a narrow
+// GEMM on CTA-pair clusters: the narrowest pair tile that covers N, and of 1, 2
+// or 4 pairs per cluster the one with the least estimated time, in units of
+// one k-block's main-loop time: waves of clusters over the SM pairs times the
+// k-blocks of a split, plus a fixed cost per tile (prologue, drain, stores)
+// and per extra cluster round of the reduction. Ties go to fewer splits.
+struct ClusterChoice {
+  int bn = 128;
+  int cs = 1;
+};
+
+static ClusterChoice choose_narrow_cluster(int64_t M, int64_t N, int64_t K, bool b_mn, int sms) {
+  ClusterChoice c;
+  c.bn = b_mn ? (N <= 128 ? 128 : N <= 256 ? 256 : N <= 384 ? 384 : 512) : (int)bn_pair_k(N);
+  const int64_t tiles = cdiv(M, 256) * cdiv(N, c.bn);
+  const int64_t kb = std::max<int64_t>(cdiv(K, 64), 1);
+  const int pairs = std::max(1, sms / 2);
+  double best = 1e300;
+  for (int cs : {1, 2, 4}) {
+    if (cs > 1 && kb < 2 * cs) break;  // at least two k-blocks per split
+    const int64_t waves = cdiv(tiles * cs, pairs);
+    const double t = (double)waves * ((double)cdiv(kb, cs) + 4.0) + (cs > 1 ? 2.0 * c.bn / 128.0 : 0.0);
+    if (t < best - 1e-9) {
+      best = t;
+      c.cs = cs;
+    }
+  }
+  return c;
+}
+
 static NarrowChoice choose_narrow(int64_t M, int64_t N, int64_t K, bool b_mn, int sms) {
   static const int kCandK[] = {64, 128, 256, 384, 512};
   static const int kCandMN[] = {128, 256, 384, 512};
@@ -151,48 +181,36 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
   if (d.dtype == DORA_BF16) {
     const double kbB = 64.0 * 2.0;  // bytes per K element pair of rows (x 64 K per k-block)
     if (op == DORA_OP_NORM) {
-      // The Gram GEMM (CTA pairs, one tile column) is small: split K over the
-      // pairs, with its fp32 partials capped at 8 MiB and at least four
-      // k-blocks per split (the finalize sums the splits one after another).
-      p.gram_bn = bn_pair_k(r);
-      const int64_t gram_max = std::max<int64_t>(
-          1, std::min<int64_t>((int64_t(8) << 20) / (r * r * 4), cdiv(d_in, 64) / 4));
-      p.gram = choose_split(cdiv(r, 256), cdiv(d_in, 64), p.sms / 2, kbB * (128 + p.gram_bn / 2.0), 0.0,
-                            (double)r * r, gram_max);
-      p.off_gram_part = take((size_t)p.gram.splits * r * r * 4);
-      // The norm GEMM runs on CTA pairs, 256 rows x the whole rank per tile.
+      // The Gram kernel (one cluster launch) writes (s/2) G as bf16 hi + lo into
+      // off_gs directly. The norm GEMM runs on CTA pairs, 256 rows x the whole
+      // rank per tile.
       p.norm_bn = bn_pair_k(r);
       p.norm = choose_split(cdiv(d_out, 256), cdiv(d_in, 64) + 2 * cdiv(r, 64), p.sms / 2,
                             kbB * (128 + p.norm_bn / 2.0), 0.0, (double)d_out);
       p.off_norm_part = take((size_t)p.norm.splits * d_out * 4);
       p.off_gs = take((size_t)r * 2 * cdiv(r, 64) * 64 * 2);
-      // split counters, one per 128-row half of a pair tile, zeroed by one memset per call
-      p.gram_tiles = 0;
+      // split counters, one per 128-row half of a pair tile, zeroed by the Gram kernel
       p.zero_bytes = (size_t)2 * cdiv(d_out, 256) * 4;
       p.off_ctr = take(p.zero_bytes);
     } else if (op == DORA_OP_FORWARD && T > 0) {
-      const NarrowChoice u = choose_narrow(T, r, d_in, false, p.sms);
+      const ClusterChoice u = choose_narrow_cluster(T, r, d_in, false, p.sms);
       p.u_bn = u.bn;
-      p.u = u.split;
-      if (p.u.splits > 1) p.off_u_part = take((size_t)p.u.splits * T * r * 4);
+      p.u_cs = u.cs;
       p.off_su = take((size_t)T * r * 2);
     } else if ((op == DORA_OP_BACKWARD || op == DORA_OP_BACKWARD_FULL) && T > 0) {
       p.off_dz = take((size_t)T * d_out * 2);
       p.dm_rowblocks = (int)cdiv(T, 256);
       p.off_dm_part = take((size_t)p.dm_rowblocks * d_out * 4);
-      const NarrowChoice du = choose_narrow(T, r, d_out, true, p.sms);
+      const ClusterChoice du = choose_narrow_cluster(T, r, d_out, true, p.sms);
       p.du_bn = du.bn;
-      p.du = du.split;
-      if (p.du.splits > 1) p.off_du_part = take((size_t)p.du.splits * T * r * 4);
+      p.du_cs = du.cs;
       p.off_du = take((size_t)T * r * 2);
-      const NarrowChoice dB = choose_narrow_1cta(d_out, r, T, true, p.sms);
+      const ClusterChoice dB = choose_narrow_cluster(d_out, r, T, true, p.sms);
       p.dB_bn = dB.bn;
-      p.dB = dB.split;
-      if (p.dB.splits > 1) p.off_dB_part = take((size_t)p.dB.splits * d_out * r * 4);
-      const NarrowChoice dA = choose_narrow_1cta(d_in, r, T, true, p.sms);
+      p.dB_cs = dB.cs;
+      const ClusterChoice dA = choose_narrow_cluster(d_in, r, T, true, p.sms);
       p.dA_bn = dA.bn;
-      p.dA = dA.split;
-      if (p.dA.splits > 1) p.off_dA_part = take((size_t)p.dA.splits * d_in * r * 4);
+      p.dA_cs = dA.cs;
       // counters of the dm column strips, zeroed by one memset per call
       p.zero_bytes = (size_t)cdiv(d_out, 64) * 4;
       p.off_ctr = take(p.zero_bytes);
@@ -200,12 +218,6 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
         const int64_t rp = cdiv(r, 64) * 64;
         p.off_kappa = take((size_t)d_out * 4);
         p.off_bk = take((size_t)d_out * r * 2);
-        p.gram_bn = bn_pair_k(r);
-        const int64_t gram_max = std::max<int64_t>(
-            1, std::min<int64_t>((int64_t(8) << 20) / (r * r * 4), cdiv(d_in, 64) / 4));
-        p.gram = choose_split(cdiv(r, 256), cdiv(d_in, 64), p.sms / 2, kbB * (128 + p.gram_bn / 2.0), 0.0,
-                              (double)r * r, gram_max);
-        p.off_gram_part = take((size_t)p.gram.splits * r * r * 4);
         p.off_gs = take((size_t)r * 2 * rp * 2);
         const NarrowChoice q = choose_narrow(d_out, r, d_in + 2 * rp, false, p.sms);
         p.q_bn = q.bn;

@@ -24,6 +24,7 @@
 
 #include "dora_internal.h"
 #include "gemm_sm100.cuh"
+#include "gram_sm100.cuh"
 #include "merge_sm100.cuh"
 
 namespace dora {
@@ -137,6 +138,7 @@ struct GemmArgs {
   int M = 0, N = 0;
   Split split;
   int a1_kwrap = 0;  // see GemmGeom::a1_kwrap
+  int defer_wait_src1 = 0;  // see GemmGeom::defer_wait_src1 (CTA-pair split kernel)
   const char* name = "gemm";
 };
 
@@ -288,6 +290,7 @@ struct EpiNorm {
     p.gm1[m] = (mi - c) / c;
   }
   static constexpr bool kReadsA = true;
+  static constexpr bool kRefillA1 = true;
   // row_ptr: this thread's 128-byte row of the swizzled W0 tile. The swizzle
   // permutes the row's eight 16-byte chunks by (row mod 8), which a sum of
   // squares does not see; reading chunk j ^ (row mod 8) at step j keeps the
@@ -306,40 +309,54 @@ struct EpiNorm {
     }
     st.ss += acc;
   }
-  // The tile's B rows [128 x r] are brought into the (now idle) stage ring by
-  // TMA through the A source-1 map, in 64-column slabs of the same swizzled
-  // layout, then dotted with the accumulator rows.
+  // The tile's B rows [128 x r] (the A source-1 operand) were prefetched by the
+  // producer into the ring stages the last k-blocks released, in 64-column
+  // slabs of the same swizzled layout (EpiCtx refill fields); each row is
+  // dotted with its accumulator row, 128 columns of TMEM in flight at a time.
+  __host__ __device__ static int refill_slabs(const Params& p) { return (p.r + 63) / 64; }
   template <int BN>
   __device__ static void run(const Params& p, RowState& st, const EpiCtx& c, const GemmGeom& g) {
+    static_assert(BN % 32 == 0, "whole 32-column chunks");
     const bool row_ok = c.m < g.M;
-    const int slabs = (p.r + 63) / 64;
-    const uint32_t bytes = (uint32_t)slabs * 16384u;
-    // All four epilogue warps are past their last stage reads before the refill.
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (c.row == 0) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive_expect_tx(c.aux_bar, bytes);
-      const int m0 = c.m - c.row;
-      for (int sl = 0; sl < slabs; ++sl) tma_load_2d(c.stage_smem + sl * 16384, c.tA1, c.aux_bar, sl * 64, m0);
-    }
     mbar_wait(c.aux_bar, 0);
     const int t = c.row & 7;
+    const int sps = c.stage_stride / 16384;
     float dot = 0.f;
-    for_each_acc_chunk<BN>(c, [&](int col, float* v) {
+#pragma unroll 1
+    for (int col0 = 0; col0 < BN; col0 += 128) {
+      constexpr int kMaxChunks = BN < 128 ? BN / 32 : 4;
+      uint32_t v[kMaxChunks][32];
+      const int nch = min(kMaxChunks, (BN - col0) / 32);
+      if (c.has_acc) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int n = col + 8 * j;
-        if (n < p.r) {
-          const int slab = n >> 6, chunk = (n & 63) >> 3;
-          const uint4 w =
-              *reinterpret_cast<const uint4*>(c.stage_smem + slab * 16384 + c.row * 128 + ((chunk ^ t) << 4));
-          float b[8];
-          unpack_bf16x8(w, b);
+        for (int q = 0; q < kMaxChunks; ++q)
+          if (q < nch) tmem_ld32_async(c.taddr + (uint32_t)(col0 + 32 * q), v[q]);
+        tmem_ld_wait();
+      } else {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) dot = fmaf(b[i], v[8 * j + i], dot);
+        for (int q = 0; q < kMaxChunks; ++q)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[q][i] = 0u;
+      }
+#pragma unroll
+      for (int q = 0; q < kMaxChunks; ++q) {
+        if (q >= nch) break;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int n = col0 + 32 * q + 8 * j;
+          if (n < p.r) {
+            const int slab = n >> 6, chunk = (n & 63) >> 3;
+            const uint8_t* base = c.stage_smem + ((c.refill_first + slab / sps) % c.ring_stages) * c.stage_stride +
+                                  (slab % sps) * 16384;
+            const uint4 w = *reinterpret_cast<const uint4*>(base + c.row * 128 + ((chunk ^ t) << 4));
+            float b[8];
+            unpack_bf16x8(w, b);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dot = fmaf(b[i], __uint_as_float(v[q][8 * j + i]), dot);
+          }
         }
       }
-    });
+    }
     const float part = fmaf(p.two_s, dot, st.ss);
     if (c.splits == 1) {
       if (row_ok) finish(p, c.m, part);
@@ -364,6 +381,7 @@ struct EpiCompose {
   };
   using RowState = NoRowState;
   static constexpr bool kReadsA = false;
+  static constexpr bool kRefillA1 = false;
   static constexpr int kStageOutBytes = 0;
   __device__ static void on_a_stage(const Params&, RowState&, const uint8_t*, bool) {}
   template <int BN>
@@ -382,7 +400,8 @@ struct EpiCompose {
           float o[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) o[i] = fmaf(gm[i], v[8 * j + i], v[8 * j + i]);
-          store_bf16x8(yrow + 8 * j, o);
+          // y is not read again inside the layer step; pre is, by the compose backward.
+          store_bf16x8_cs(yrow + 8 * j, o);
           if (p.pre) store_bf16x8(p.pre + (long long)c.m * p.ldo + n + 8 * j, v + 8 * j);
         }
       }
@@ -400,6 +419,7 @@ struct EpiAxpyBF16 {
   };
   using RowState = NoRowState;
   static constexpr bool kReadsA = false;
+  static constexpr bool kRefillA1 = false;
   static constexpr int kStageOutBytes = 0;
   __device__ static void on_a_stage(const Params&, RowState&, const uint8_t*, bool) {}
   template <int BN>
@@ -444,7 +464,7 @@ static cudaError_t launch_gemm_pair_split(const GemmArgs& g, const typename Epi:
     tb1 = tb0;
   }
   const int kps = g.split.kb_per_split > 0 ? g.split.kb_per_split : kb0 + kb1;
-  GemmGeom geom{g.M, g.N, kb0, kb1, kps, g.a1_kwrap};
+  GemmGeom geom{g.M, g.N, kb0, kb1, kps, g.a1_kwrap, g.defer_wait_src1};
   const long long splits = ceil_div(std::max(kb0 + kb1, 1), kps);
   const long long tiles = ceil_div(g.N, Cfg::BN) * ceil_div(g.M, 2 * kBM);
   auto kern = gemm_sm100_pair_split_kernel<Cfg, Epi>;
@@ -515,45 +535,6 @@ __global__ void reduce_splits_bf16_kernel(const float* __restrict__ part, int sp
 #pragma unroll
       for (int j = 0; j < 4; ++j) out[(long long)(n + j) * ldo + m] = __float2bfloat16_rn(o[j]);
     }
-  }
-}
-
-// Gram finalize: x = scale sum_z part[z] in fp32 (split order fixed), written
-// as two bf16 halves Gs2[n] = [hi(x_n,0..r-1), 0 .. | lo(x_n,0..r-1), 0 ..]
-// with rp columns each, hi = bf16(x) and lo = bf16(x - hi), so hi + lo carries
-// x to about 2^-17. Each thread takes 4 consecutive columns of one half-row.
-__global__ void gram_finalize_kernel(const float* __restrict__ part, int splits, int r, int rp, float scale,
-                                     __nv_bfloat16* __restrict__ gs2) {
-  pdl_trigger();
-  pdl_wait();
-  const int qn = rp / 4;  // 4-column groups per half-row
-  const long long total = (long long)r * 2 * qn;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const int n = (int)(i / (2 * qn));
-    const int qq = (int)(i % (2 * qn));
-    const bool lo = qq >= qn;
-    const int c = (lo ? qq - qn : qq) * 4;
-    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (c < r) {
-      const float* src = part + (long long)n * r + c;
-#pragma unroll 4
-      for (int z = 0; z < splits; ++z) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(src + (long long)z * r * r));
-        x.x += v.x;
-        x.y += v.y;
-        x.z += v.z;
-        x.w += v.w;
-      }
-    }
-    const float xs[4] = {scale * x.x, scale * x.y, scale * x.z, scale * x.w};
-    __nv_bfloat16 o[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const __nv_bfloat16 hi = __float2bfloat16_rn(xs[j]);
-      o[j] = (c + j < r) ? (lo ? __float2bfloat16_rn(xs[j] - __bfloat162float(hi)) : hi) : __float2bfloat16_rn(0.f);
-    }
-    *reinterpret_cast<uint2*>(gs2 + (long long)n * 2 * rp + (lo ? rp : 0) + c) = *reinterpret_cast<const uint2*>(o);
   }
 }
 
@@ -732,62 +713,156 @@ static cudaError_t narrow_gemm_1cta(int bn, const GemmArgs& g, float alpha, __nv
   return reduce_splits(part, g.split, sstride, g.M, g.N, alpha, out, ldo, transpose, reduce_name, st);
 }
 
-template <bool A_MN, bool B_MN>
-static cudaError_t narrow_gemm_pair(int bn, const GemmArgs& g, float alpha, __nv_bfloat16* out, long long ldo,
-                                    bool transpose, float* part, const char* reduce_name, int sms, cudaStream_t st) {
-  if (g.split.splits == 1) {
-    EpiStoreBF16::Params p{out, ldo, alpha, transpose ? 1 : 0};
-    return pair_gemm_bn<A_MN, B_MN, EpiStoreBF16>(bn, g, p, sms, st);
+// Narrow GEMM on CTA-pair clusters (gemm_sm100_pair_cluster_kernel): out =
+// alpha * A B^T in bf16, the K splits of each tile reduced inside its cluster.
+template <class Cfg, int CS>
+static cudaError_t launch_pair_cluster(const GemmArgs& g, const NarrowOut& o, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  t_detail.clear();
+  if (!make_map(&ta, g.a0, Cfg::A_MN ? 64 : kBM, "A") || !make_map(&tb, g.b0, Cfg::B_MN ? 64 : Cfg::B_BOX, "B"))
+    return cudaErrorInvalidValue;
+  const int kb = (int)std::max<int64_t>(ceil_div(g.K0, kBK), 1);
+  GemmGeom geom{g.M, g.N, kb, 0, (int)ceil_div(kb, CS), 0, 0};
+  const long long tiles = ceil_div(g.N, Cfg::BN) * ceil_div(g.M, 2 * kBM);
+  auto kern = gemm_sm100_pair_cluster_kernel<Cfg, CS>;
+  constexpr int smem_bytes = PairClusterLayout<Cfg>::SMEM_BYTES;
+  static std::atomic<unsigned long long> smem_set{0};
+  cudaError_t e = set_smem_once(smem_set, kern, smem_bytes);
+  if (e != cudaSuccess) {
+    t_detail = "shared-memory attribute (" + std::to_string(smem_bytes) + " bytes)";
+    return e;
   }
-  EpiPartialTMA::Params p;
-  if (!make_map_f32_3d(&p.map, part, g.N, g.M, g.split.splits, 32, 32)) return cudaErrorInvalidValue;
-  cudaError_t e = pair_gemm_bn<A_MN, B_MN, EpiPartialTMA>(bn, g, p, sms, st);
-  if (e != cudaSuccess) return e;
-  const long long sstride = (long long)g.M * g.N;
-  return reduce_splits(part, g.split, sstride, g.M, g.N, alpha, out, ldo, transpose, reduce_name, st);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * CS * tiles));
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = smem_bytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2 * CS;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  {
+    ProfRange pr(g.name, st);
+    e = cudaLaunchKernelEx(&cfg, kern, ta, tb, geom, o);
+  }
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess)
+    t_detail = "pair cluster launch, " + std::to_string(tiles) + " tiles x " + std::to_string(CS) + " pairs";
+  return e;
+}
+
+template <int BN, bool A_MN, bool B_MN>
+static cudaError_t pair_cluster_cs(int cs, const GemmArgs& g, const NarrowOut& o, cudaStream_t st) {
+  using Cfg = PairCfg<BN, A_MN, B_MN>;
+  if (cs == 1) return launch_pair_cluster<Cfg, 1>(g, o, st);
+  if (cs == 2) return launch_pair_cluster<Cfg, 2>(g, o, st);
+  if (cs == 4) return launch_pair_cluster<Cfg, 4>(g, o, st);
+  t_detail = "no cluster of " + std::to_string(cs) + " pairs";
+  return cudaErrorInvalidValue;
+}
+
+template <bool A_MN, bool B_MN>
+static cudaError_t narrow_cluster(int bn, int cs, const GemmArgs& g, float alpha, __nv_bfloat16* out, long long ldo,
+                                  bool transpose, cudaStream_t st) {
+  const NarrowOut o{out, ldo, alpha, transpose ? 1 : 0};
+  if constexpr (!B_MN) {
+    if (bn == 64) return pair_cluster_cs<64, A_MN, B_MN>(cs, g, o, st);
+  }
+  if (bn == 128) return pair_cluster_cs<128, A_MN, B_MN>(cs, g, o, st);
+  if (bn == 256) return pair_cluster_cs<256, A_MN, B_MN>(cs, g, o, st);
+  if (bn == 384) return pair_cluster_cs<384, A_MN, B_MN>(cs, g, o, st);
+  if (bn == 512) return pair_cluster_cs<512, A_MN, B_MN>(cs, g, o, st);
+  t_detail = "no pair cluster tile of width " + std::to_string(bn);
+  return cudaErrorInvalidValue;
 }
 
 // ============================================================== operations
 
-// Gram G = A A^T (CTA pairs, split K into fp32 partials), then scale * G as
-// bf16 hi and lo halves [r x 2 rp] for a K-extension of a later GEMM.
-static cudaError_t gram_hi_lo(const dora_desc_t& d, const Plan& p, const void* A, float scale, float* gram_part,
-                              __nv_bfloat16* gs, cudaStream_t st) {
+// Gs = scale * A A^T as bf16 hi and lo halves [r x 2 rp] for a K-extension of a
+// later GEMM, in one cluster launch (gram_sm100.cuh). zero_words (may be null)
+// are zeroed by the kernel before the next kernel is allowed to start.
+// spare_sms: SMs the next kernel leaves free; when the Gram's tiles fit there
+// with two or more CTAs each, it takes as many CTAs per tile as fit (it then
+// runs beside the next kernel), else eight.
+template <int CS>
+static cudaError_t launch_gram_cs(const CUtensorMap& ta, const GramParams& gp0, int tiles, cudaStream_t st) {
+  GramParams gp = gp0;
+  gp.kps = (int)ceil_div(gp.kb_total, CS);
+  auto kern = gram_cluster_kernel<CS>;
+  static std::atomic<unsigned long long> smem_set{0};
+  cudaError_t e = set_smem_once(smem_set, kern, kGramSmemBytes);
+  if (e != cudaSuccess) {
+    t_detail = "Gram shared-memory attribute";
+    return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CS, (unsigned)tiles);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = kGramSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = CS;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  {
+    ProfRange pr("gram_gemm", st);
+    e = cudaLaunchKernelEx(&cfg, kern, ta, gp);
+  }
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess)
+    t_detail = "Gram cluster launch, " + std::to_string(tiles) + " tiles x " + std::to_string(CS) + " CTAs";
+  return e;
+}
+
+static cudaError_t launch_gram(const dora_desc_t& d, const void* A, float scale, __nv_bfloat16* gs,
+                               unsigned int* zero_words, int zero_count, int spare_sms, cudaStream_t st) {
   const int r = (int)d.r, d_in = (int)d.d_in;
-  const int rp = (int)ceil_div(r, kBK) * kBK;
-  GemmArgs ga;
-  ga.a0 = Mat{A, r, d_in, d_in};
-  ga.b0 = ga.a0;
-  ga.K0 = d_in;
-  ga.M = r;
-  ga.N = r;
-  ga.split = p.gram;
-  ga.name = "gram_gemm";
-  EpiPartialTMA::Params pp;
-  if (!make_map_f32_3d(&pp.map, gram_part, r, r, p.gram.splits, 32, 32)) return cudaErrorInvalidValue;
-  cudaError_t e = pair_gemm_bn<false, false, EpiPartialTMA>(p.gram_bn, ga, pp, p.sms, st);
-  if (e != cudaSuccess) return e;
-  const long long total = (long long)r * 2 * (rp / 4);
-  ProfRange pr("gram_finalize", st);
-  e = launch_pdl(gram_finalize_kernel, dim3((unsigned)std::min<long long>(ceil_div(total, 256), 2048)), dim3(256), 0,
-                 st, (const float*)gram_part, p.gram.splits, r, rp, scale, gs);
-  return e == cudaSuccess ? cudaGetLastError() : e;
+  CUtensorMap ta;
+  t_detail.clear();
+  if (!make_map(&ta, Mat{A, r, d_in, d_in}, kGramTile, "A (Gram)")) return cudaErrorInvalidValue;
+  GramParams gp;
+  gp.r = r;
+  gp.rp = (int)ceil_div(r, kBK) * kBK;
+  gp.nt = (int)ceil_div(r, kGramTile);
+  gp.kb_total = (int)ceil_div(d_in, kBK);
+  gp.kps = 0;
+  gp.scale = scale;
+  gp.gs2 = gs;
+  gp.zero_words = zero_words;
+  gp.zero_count = zero_count;
+  const int tiles = gp.nt * (gp.nt + 1) / 2;
+  int cs = 8;
+  if (2 * tiles <= spare_sms) cs = 8 * tiles <= spare_sms ? 8 : 4 * tiles <= spare_sms ? 4 : 2;
+  switch (cs) {
+    case 2: return launch_gram_cs<2>(ta, gp, tiles, st);
+    case 4: return launch_gram_cs<4>(ta, gp, tiles, st);
+    default: return launch_gram_cs<8>(ta, gp, tiles, st);
+  }
 }
 
 dora_status_t bf16_norm(const dora_desc_t& d, const Plan& p, const void* W0, const void* A, const void* B,
                         const float* m, float* C, float* g, float* gm1, uint8_t* ws, cudaStream_t st) {
   const int r = (int)d.r, d_in = (int)d.d_in, d_out = (int)d.d_out;
-  float* gram_part = reinterpret_cast<float*>(ws + p.off_gram_part);
   __nv_bfloat16* gs = reinterpret_cast<__nv_bfloat16*>(ws + p.off_gs);
   float* norm_part = reinterpret_cast<float*>(ws + p.off_norm_part);
   unsigned int* ctr = reinterpret_cast<unsigned int*>(ws + p.off_ctr);
-  // The norm's split counters start at zero.
-  cudaError_t e = cudaMemsetAsync(ws + p.off_ctr, 0, p.zero_bytes, st);
-  if (e != cudaSuccess) return cuda_status(e, "dora_norm: clearing counters");
 
-  // Gram G = A A^T in fp32 partials, then (s/2) G as bf16 hi and lo halves.
+  // (s/2) G as bf16 hi and lo halves; the same kernel zeroes the norm's split counters.
   const int rp = (int)ceil_div(r, kBK) * kBK;
-  e = gram_hi_lo(d, p, A, 0.5f * d.s, gram_part, gs, st);
+  // SMs the norm GEMM leaves free (one CTA pair per tile and K split, at most one per SM pair).
+  const long long norm_pairs = ceil_div(d_out, 2 * kBM) * p.norm.splits;
+  const int spare = p.sms - 2 * (int)std::min<long long>(norm_pairs, p.sms / 2);
+  cudaError_t e = launch_gram(d, A, 0.5f * d.s, gs, ctr, (int)(p.zero_bytes / 4), spare, st);
   if (e != cudaSuccess) return gemm_status(e, "dora_norm: Gram");
 
   // acc = [W0 | B | B] [A | Gs_hi | Gs_lo]^T with the factored-norm epilogue,
@@ -803,9 +878,10 @@ dora_status_t bf16_norm(const dora_desc_t& d, const Plan& p, const void* W0, con
   na.M = d_out;
   na.N = r;
   na.split = p.norm;
+  na.defer_wait_src1 = 1;  // only Gs comes from the Gram kernel: stream W0 while it runs
   na.name = "norm_gemm";
-  EpiNorm::Params np{reinterpret_cast<const __nv_bfloat16*>(B), r, 2.0f * d.s, norm_part, d_out,
-                     ctr + p.gram_tiles, m, C, g, gm1};
+  EpiNorm::Params np{reinterpret_cast<const __nv_bfloat16*>(B), r, 2.0f * d.s, norm_part, d_out, ctr, m, C, g,
+                     gm1};
   e = norm_gemm(p.norm_bn, na, np, st);
   return gemm_status(e, "dora_norm: factored norm GEMM");
 }
@@ -825,10 +901,8 @@ dora_status_t bf16_forward(const dora_desc_t& d, const Plan& p, int64_t T, const
   ua.K0 = d_in;
   ua.M = Ti;
   ua.N = r;
-  ua.split = p.u;
   ua.name = "u_gemm";
-  cudaError_t e = narrow_gemm_pair<false, false>(p.u_bn, ua, d.s, su, r, false, reinterpret_cast<float*>(ws + p.off_u_part),
-                                "u_reduce", p.sms, st);
+  cudaError_t e = narrow_cluster<false, false>(p.u_bn, p.u_cs, ua, d.s, su, r, false, st);
   if (e != cudaSuccess) return gemm_status(e, "dora_forward: LoRA down projection");
 
   // pre = [x | su] [W0 | B]^T, y = pre + gm1 * pre
@@ -918,10 +992,8 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.K0 = d_out;
     a.M = Ti;
     a.N = r;
-    a.split = p.du;
     a.name = "du_gemm";
-    cudaError_t e = narrow_gemm_pair<false, true>(p.du_bn, a, d.s, du, r, false,
-                                             reinterpret_cast<float*>(ws + p.off_du_part), "du_reduce", p.sms, st);
+    cudaError_t e = narrow_cluster<false, true>(p.du_bn, p.du_cs, a, d.s, du, r, false, st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: du");
   }
   // dB = dz^T su  (both token-major: K = T)
@@ -932,10 +1004,9 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.K0 = Ti;
     a.M = d_out;
     a.N = r;
-    a.split = p.dB;
     a.name = "dB_gemm";
-    cudaError_t e = narrow_gemm_1cta<true, true>(p.dB_bn, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dB), r, false,
-                                                 reinterpret_cast<float*>(ws + p.off_dB_part), "dB_reduce", st);
+    cudaError_t e = narrow_cluster<true, true>(p.dB_bn, p.dB_cs, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dB), r,
+                                               false, st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: dB");
   }
   // dA^T = x^T du, stored transposed into dA [r x d_in]
@@ -946,10 +1017,9 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.K0 = Ti;
     a.M = d_in;
     a.N = r;
-    a.split = p.dA;
     a.name = "dA_gemm";
-    cudaError_t e = narrow_gemm_1cta<true, true>(p.dA_bn, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dA), d_in,
-                                                 true, reinterpret_cast<float*>(ws + p.off_dA_part), "dA_reduce", st);
+    cudaError_t e = narrow_cluster<true, true>(p.dA_bn, p.dA_cs, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dA), d_in,
+                                               true, st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: dA");
   }
   // dx = [dz | du] [W0 ; A]  (W0 and A read MN-major: K rows, N = d_in contiguous)
@@ -1000,7 +1070,7 @@ dora_status_t bf16_backward_full(const dora_desc_t& d, const Plan& p, int64_t T,
     if (e != cudaSuccess) return cuda_status(e, "dora_backward_full: kappa");
   }
   // s G as bf16 hi + lo, then Q = W0 A^T + s B G into fp32 split partials.
-  e = gram_hi_lo(d, p, A, d.s, reinterpret_cast<float*>(ws + p.off_gram_part), gs, st);
+  e = launch_gram(d, A, d.s, gs, nullptr, 0, 0, st);
   if (e != cudaSuccess) return gemm_status(e, "dora_backward_full: Gram");
   {
     GemmArgs a;

@@ -22,27 +22,24 @@ struct Split {
 struct Plan {
   int sms = 148;
   // norm
-  Split gram, norm;
-  int gram_bn = 0, norm_bn = 0;
-  size_t off_gram_part = 0, off_gs = 0, off_norm_part = 0;
-  // forward
-  Split u;
-  int u_bn = 0;
-  size_t off_u_part = 0, off_su = 0;
-  // backward
+  Split norm;
+  int norm_bn = 0;
+  size_t off_gs = 0, off_norm_part = 0;
+  // forward: u = s x A^T on CTA-pair clusters (tile width, pairs per cluster = K splits)
+  int u_bn = 0, u_cs = 1;
+  size_t off_su = 0;
+  // backward: du, dB, dA likewise
   int dm_rowblocks = 0;
-  Split du, dB, dA;
-  int du_bn = 0, dB_bn = 0, dA_bn = 0;
-  size_t off_dz = 0, off_dm_part = 0, off_du_part = 0, off_du = 0, off_dB_part = 0, off_dA_part = 0;
+  int du_bn = 0, du_cs = 1, dB_bn = 0, dB_cs = 1, dA_bn = 0, dA_cs = 1;
+  size_t off_dz = 0, off_dm_part = 0, off_du = 0;
   // full (non-detached) gradient: kappa, kappa-scaled B, Gram, Q = W' A^T, H = s B^T diag(kappa) B
   Split q, h;
   int q_bn = 0, h_bn = 0;
   size_t off_kappa = 0, off_bk = 0, off_q_part = 0, off_h_part = 0, off_h = 0;
   // DVoRA gradient: row blocks of the dd partial sums (scratch in off_f32_a)
   int vera_blocks = 0;
-  // split counters (+ padding that must start at zero), cleared by one memset per call
+  // split counters (+ padding that must start at zero), cleared once per call
   size_t off_ctr = 0, zero_bytes = 0;
-  int gram_tiles = 0;
   // fp32 path scratch
   size_t off_f32_a = 0, off_f32_b = 0, off_f32_c = 0;
   size_t total = 0;

@@ -37,6 +37,11 @@ struct GemmGeom {
   int kb1;           // k-blocks taken from source 1
   int kb_per_split;  // k-blocks per blockIdx.z
   int a1_kwrap;      // > 0: source-1 A coordinates wrap modulo this many K elements
+  // CTA-pair split kernel only: nonzero when only the source-1 operands come from
+  // the preceding grid. The kernel then starts its source-0 main loop at once;
+  // the producer waits for the preceding grid just before its first source-1
+  // load, and the epilogue warps before they write anything.
+  int defer_wait_src1 = 0;
 };
 
 template <int BN_, bool A_MN_, bool B_MN_>
@@ -77,6 +82,13 @@ struct EpiCtx {
   int stage_bytes;            // bytes of the ring
   uint64_t* aux_bar;          // spare mbarrier (count 1), phase 0 unused so far
   const CUtensorMap* tA1;     // A-operand source-1 tensor map
+  // CTA-pair split kernel with an epilogue that has its A source-1 rows
+  // prefetched (Epi::kRefillA1): 16 KB slab sl sits in ring stage
+  // (refill_first + sl / (stage_stride / 16384)) % ring_stages, at
+  // (sl % (stage_stride / 16384)) * 16384 bytes, complete on aux_bar phase 0.
+  int refill_first;
+  int ring_stages;
+  int stage_stride;
   // K-split bookkeeping (non-persistent kernels): the output rows' index (one
   // per 128-row block), the number of splits, and a shared-memory word for
   // the last-split decision.
@@ -84,6 +96,25 @@ struct EpiCtx {
   int splits;
   uint32_t* flag;
 };
+
+__device__ __forceinline__ void store_bf16x8(__nv_bfloat16* dst, const float* v) {
+  __nv_bfloat162 p[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) p[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+  *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(p);
+}
+
+// The same with the streaming (evict-first) cache hint: for outputs no kernel
+// of the call reads again, so that their lines leave L2 early and make room
+// for the data the next kernel reads.
+__device__ __forceinline__ void store_bf16x8_cs(__nv_bfloat16* dst, const float* v) {
+  __nv_bfloat162 p[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) p[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+  const uint4 w = *reinterpret_cast<const uint4*>(p);
+  asm volatile("st.global.cs.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "r"(w.x), "r"(w.y), "r"(w.z), "r"(w.w)
+               : "memory");
+}
 
 // 16-column TMEM load (for tiles whose width is an odd multiple of 16).
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
@@ -280,6 +311,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     c.stage_bytes = STAGES * Cfg::STAGE_BYTES;
     c.aux_bar = aux;
     c.tA1 = &tA1;
+    c.refill_first = nkb;
+    c.ring_stages = STAGES;
+    c.stage_stride = Cfg::STAGE_BYTES;
     c.tile_id = m_tile * (int)gridDim.x + n_tile;
     c.splits = (int)gridDim.z;
     c.flag = tmem_slot + 1;
@@ -555,6 +589,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       c.stage_bytes = EPI_BYTES;
       c.aux_bar = nullptr;
       c.tA1 = &tA1;
+      c.refill_first = 0;
+      c.ring_stages = 0;
+      c.stage_stride = 0;
       c.tile_id = t;
       c.splits = splits;
       c.flag = nullptr;
@@ -654,23 +691,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   pdl_trigger();
-  pdl_wait();
+  const bool defer = geom.defer_wait_src1 != 0;
+  if (!defer) pdl_wait();
 
   const int m0 = tm * 2 * kBM + (int)rank * kBM;
   if (warp == 0) {
     if (lane == 0) {
       const int nb0 = tn * Cfg::BN + (int)rank * Cfg::H0;
       const int nb1 = tn * Cfg::BN + Cfg::N0 + (int)rank * Cfg::H1;
+      bool waited = !defer;
+      bool ok = true;
 #pragma unroll 1
       for (int i = 0; i < nkb; ++i) {
         const int s = i % STAGES;
-        if (!mbar_wait(&empty[s], ((uint32_t)(i / STAGES) & 1u) ^ 1u)) break;
+        if (!mbar_wait(&empty[s], ((uint32_t)(i / STAGES) & 1u) ^ 1u)) {
+          ok = false;
+          break;
+        }
         uint8_t* sa = smem + s * Cfg::STAGE_BYTES;
         uint8_t* sb = sa + Cfg::A_BYTES;
         const uint32_t fb = mapa_shared(smem_u32(&full[s]), 0);
-        if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
         const int kb = kb_begin + i;
         const bool src1 = kb >= geom.kb0;
+        if (src1 && !waited) {
+          pdl_wait();  // the source-1 operands come from the preceding grid
+          waited = true;
+        }
+        if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
         const int k0 = (src1 ? kb - geom.kb0 : kb) * kBK;
         const int k0a = (src1 && geom.a1_kwrap > 0) ? k0 % geom.a1_kwrap : k0;
         const CUtensorMap* ta = src1 ? &tA1 : &tA0;
@@ -694,6 +741,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             tma_load_2d_pair(sb + Cfg::B1_OFFSET + j * Cfg::B_BOX * 128, tb, fb, k0, nb1 + j * Cfg::B_BOX);
           else
             tma_load_2d_pair(sb + Cfg::B1_OFFSET + j * 8192, tb, fb, nb1 + j * 64, k0);
+        }
+      }
+      if constexpr (Epi::kRefillA1) {
+        // The epilogue's rows of the A source-1 operand (this CTA's 128 rows, 64-column
+        // slabs of 16 KB), loaded into the ring stages as the last k-blocks release
+        // them, so they arrive while the final MMAs still run.
+        constexpr int kSps = Cfg::STAGE_BYTES / 16384;
+        static_assert(kSps >= 1 && (Cfg::BN / 64 + kSps - 1) / kSps <= STAGES, "refill fits the ring");
+        const int slabs = Epi::refill_slabs(ep);
+        if (ok && slabs > 0) {
+          mbar_arrive_expect_tx(aux, (uint32_t)slabs * 16384u);
+          for (int sl = 0; sl < slabs; ++sl) {
+            const int u = nkb + sl / kSps;
+            const int s = u % STAGES;
+            if (sl % kSps == 0 && !mbar_wait(&empty[s], ((uint32_t)(u / STAGES) & 1u) ^ 1u)) break;
+            tma_load_2d(smem + s * Cfg::STAGE_BYTES + (sl % kSps) * 16384, &tA1, aux, sl * 64, m0);
+          }
         }
       }
     }
@@ -743,6 +807,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
     mbar_wait(accf, 0);
     tc_fence_after();
+    if (defer) pdl_wait();  // before the epilogue writes anything
     EpiCtx c;
     c.taddr = tmem + ((uint32_t)(q * 32) << 16);
     c.row = row;
@@ -754,6 +819,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     c.stage_bytes = STAGES * Cfg::STAGE_BYTES;
     c.aux_bar = aux;
     c.tA1 = &tA1;
+    c.refill_first = nkb;
+    c.ring_stages = STAGES;
+    c.stage_stride = Cfg::STAGE_BYTES;
     c.tile_id = (tm * 2 + (int)rank) * n_tiles + tn;
     c.splits = (int)gridDim.z;
     c.flag = tmem_slot + 1;
@@ -769,14 +837,275 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-// ------------------------------------------------------------------ epilogues
+// ------------------------------------------------------------------ CTA-pair cluster split-K variant
+//
+// For narrow GEMMs (N = the LoRA rank, long K) whose output tiles are too few
+// to fill the GPU: a cluster of 2 * CS CTAs, i.e. CS CTA pairs, computes one
+// 256 x BN output tile, pair z (cluster ranks 2z and 2z + 1) taking the z-th
+// K range. Each pair runs the pair kernels' main loop (its leader is rank 2z;
+// commits go to the pair's two CTAs). The accumulators are then reduced inside
+// the cluster, CW columns at a time: every CTA drains its 128 TMEM rows into
+// its own shared memory (the idle stage ring), and after a cluster barrier
+// CTA (z, q) sums rows [z * 128 / CS, (z + 1) * 128 / CS) of half q over the
+// cluster's CS CTAs of that half, always in split order, by reading their
+// buffers through distributed shared memory, then scales by alpha and stores
+// bf16 (row-major, or transposed out[n][m]). No fp32 partials reach global
+// memory and the result does not depend on timing.
 
-__device__ __forceinline__ void store_bf16x8(__nv_bfloat16* dst, const float* v) {
-  __nv_bfloat162 p[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) p[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-  *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(p);
+struct NarrowOut {
+  __nv_bfloat16* out;
+  long long ldo;  // row length of out (elements)
+  float alpha;
+  int transpose;  // 0: out[m][n]; 1: out[n][m]
+};
+
+template <class Cfg>
+struct PairClusterLayout {
+  static constexpr int STAGES_RAW = kSmemBudget / Cfg::STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static_assert(STAGES >= 2, "stages");
+  static constexpr int CW = Cfg::BN < 256 ? Cfg::BN : 256;  // columns reduced per round
+  static constexpr int RS = CW + 4;                         // fp32 row stride of the reduction buffer
+  static_assert(Cfg::BN % CW == 0 || Cfg::BN == 384, "whole rounds");
+  static_assert(128 * RS * 4 <= STAGES * Cfg::STAGE_BYTES, "reduction buffer fits the ring");
+  static constexpr int SMEM_BYTES = STAGES * Cfg::STAGE_BYTES + Cfg::BAR_BYTES + 1024;
+};
+
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t cluster_addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+  return v;
 }
+
+__device__ __forceinline__ float4 ld_dsmem_v4(uint32_t cluster_addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(cluster_addr)
+               : "memory");
+  return v;
+}
+
+template <class Cfg, int CS>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_sm100_pair_cluster_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tB,
+                                   const GemmGeom geom, const NarrowOut o) {
+  static_assert(CS == 1 || CS == 2 || CS == 4, "pairs per cluster");
+  using L = PairClusterLayout<Cfg>;
+  constexpr int STAGES = L::STAGES;
+  constexpr int CW = L::CW;
+  constexpr int RS = L::RS;
+  constexpr int ROWS = 128 / CS;  // rows of its half each CTA reduces
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accf = empty + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  float* red = reinterpret_cast<float*>(smem);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t crank = cluster_ctarank();
+  const uint32_t q = crank & 1u;              // half of the 256-row tile
+  const int z = (int)(crank >> 1);            // K split
+  const uint32_t leader = crank & ~1u;
+  const uint16_t pair_mask = (uint16_t)(3u << leader);
+  const int n_tiles = (geom.N + Cfg::BN - 1) / Cfg::BN;
+  const int t = blockIdx.x / (2 * CS);
+  const int tm = t / n_tiles, tn = t - tm * n_tiles;
+  const int kb_total = geom.kb0;
+  const int kb_begin = z * geom.kb_per_split;
+  const int kb_end = min(kb_total, kb_begin + geom.kb_per_split);
+  const int nkb = kb_end > kb_begin ? kb_end - kb_begin : 0;
+  const int m0 = tm * 2 * kBM + (int)q * kBM;
+
+  if (threadIdx.x == 0) {
+#pragma unroll 1
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accf, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tA);
+    prefetch_tmap(&tB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, Cfg::ACC_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_trigger();
+  pdl_wait();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const int nb0 = tn * Cfg::BN + (int)q * Cfg::H0;
+      const int nb1 = tn * Cfg::BN + Cfg::N0 + (int)q * Cfg::H1;
+#pragma unroll 1
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % STAGES;
+        if (!mbar_wait(&empty[s], ((uint32_t)(i / STAGES) & 1u) ^ 1u)) break;
+        uint8_t* sa = smem + s * Cfg::STAGE_BYTES;
+        uint8_t* sb = sa + Cfg::A_BYTES;
+        const uint32_t fb = mapa_shared(smem_u32(&full[s]), leader);
+        if (q == 0) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
+        const int k0 = (kb_begin + i) * kBK;
+        if (!Cfg::A_MN) {
+          tma_load_2d_pair(sa, &tA, fb, k0, m0);
+        } else {
+          tma_load_2d_pair(sa, &tA, fb, m0, k0);
+          tma_load_2d_pair(sa + 8192, &tA, fb, m0 + 64, k0);
+        }
+#pragma unroll
+        for (int j = 0; j < Cfg::B0_LOADS; ++j) {
+          if (!Cfg::B_MN)
+            tma_load_2d_pair(sb + j * Cfg::B_BOX * 128, &tB, fb, k0, nb0 + j * Cfg::B_BOX);
+          else
+            tma_load_2d_pair(sb + j * 8192, &tB, fb, nb0 + j * 64, k0);
+        }
+#pragma unroll
+        for (int j = 0; j < Cfg::B1_LOADS; ++j) {
+          if (!Cfg::B_MN)
+            tma_load_2d_pair(sb + Cfg::B1_OFFSET + j * Cfg::B_BOX * 128, &tB, fb, k0, nb1 + j * Cfg::B_BOX);
+          else
+            tma_load_2d_pair(sb + Cfg::B1_OFFSET + j * 8192, &tB, fb, nb1 + j * 64, k0);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && q == 0) {
+      constexpr uint32_t idesc0 = idesc_bf16_f32(2 * kBM, Cfg::N0, Cfg::A_MN, Cfg::B_MN);
+      constexpr uint32_t idesc1 = idesc_bf16_f32(2 * kBM, Cfg::N1 > 0 ? Cfg::N1 : 16, Cfg::A_MN, Cfg::B_MN);
+      constexpr uint32_t a_kstep = Cfg::A_MN ? 2048u : 32u;
+      constexpr uint32_t b_kstep = Cfg::B_MN ? 2048u : 32u;
+      constexpr uint32_t a_lbo = Cfg::A_MN ? 8192u : 16u;
+      constexpr uint32_t b_lbo = Cfg::B_MN ? 8192u : 16u;
+#pragma unroll 1
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % STAGES;
+        if (!mbar_wait(&full[s], (uint32_t)(i / STAGES) & 1u)) break;
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + s * Cfg::STAGE_BYTES);
+        const uint32_t sb = sa + Cfg::A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(sa + kk * a_kstep, a_lbo, 1024u);
+          const uint64_t bd0 = sdesc_sw128(sb + kk * b_kstep, b_lbo, 1024u);
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+          umma_bf16_pair(tmem, ad, bd0, idesc0, acc);
+          if (Cfg::N1 > 0) {
+            const uint64_t bd1 = sdesc_sw128(sb + Cfg::B1_OFFSET + kk * b_kstep, b_lbo, 1024u);
+            umma_bf16_pair(tmem + (uint32_t)Cfg::N0, ad, bd1, idesc1, acc);
+          }
+        }
+        umma_commit_pair(&empty[s], pair_mask);
+      }
+      umma_commit_pair(accf, pair_mask);
+    }
+    __syncwarp();
+  }
+
+  // ---- reduction inside the cluster, CW columns per round
+  bool acc_ok = true;
+  if (warp >= 2) {
+    // tcgen05.ld is warp-collective: the whole warp takes the same branch below.
+    acc_ok = __all_sync(0xffffffffu, mbar_wait(accf, 0));
+    tc_fence_after();
+  }
+  const uint32_t red_base = smem_u32(red);
+  const int row_lo = z * ROWS;
+#pragma unroll 1
+  for (int c0 = 0; c0 < Cfg::BN; c0 += CW) {
+    const int cw = min(CW, Cfg::BN - c0);
+    if (warp >= 2) {
+      const int qq = warp & 3;
+      const int row = qq * 32 + lane;
+      float* dst = red + row * RS;
+#pragma unroll 1
+      for (int col = 0; col < cw; col += 32) {
+        float v[32];
+        if (nkb > 0 && acc_ok) {
+          tmem_ld32(tmem + ((uint32_t)(qq * 32) << 16) + (uint32_t)(c0 + col), v);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(dst + col + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      }
+    }
+    tc_fence_before();
+    cluster_sync();  // every CTA's round is in its buffer
+    if (!o.transpose) {
+      // item = (row, 8 columns): out[m][n .. n + 7]
+      const int per_row = cw / 8;
+      for (int it = threadIdx.x; it < ROWS * per_row; it += kGemmThreads) {
+        const int lr = row_lo + it / per_row;
+        const int lc = (it % per_row) * 8;
+        const uint32_t off = (uint32_t)((lr * RS + lc) * 4);
+        float a[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a[i] = 0.f;
+#pragma unroll
+        for (int zz = 0; zz < CS; ++zz) {
+          const uint32_t src = mapa_shared(red_base + off, (uint32_t)(2 * zz) + q);
+          const float4 x0 = ld_dsmem_v4(src), x1 = ld_dsmem_v4(src + 16);
+          a[0] += x0.x; a[1] += x0.y; a[2] += x0.z; a[3] += x0.w;
+          a[4] += x1.x; a[5] += x1.y; a[6] += x1.z; a[7] += x1.w;
+        }
+        const int m = m0 + lr;
+        const int n = tn * Cfg::BN + c0 + lc;
+        if (m < geom.M && n < geom.N) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) a[i] *= o.alpha;
+          store_bf16x8(o.out + (long long)m * o.ldo + n, a);
+        }
+      }
+    } else {
+      // item = (column, 8 rows): out[n][m .. m + 7]
+      for (int it = threadIdx.x; it < (ROWS / 8) * cw; it += kGemmThreads) {
+        const int lc = it % cw;
+        const int lr = row_lo + (it / cw) * 8;
+        float a[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a[i] = 0.f;
+#pragma unroll
+        for (int zz = 0; zz < CS; ++zz) {
+          const uint32_t src = mapa_shared(red_base + (uint32_t)((lr * RS + lc) * 4), (uint32_t)(2 * zz) + q);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) a[i] += ld_dsmem_f32(src + (uint32_t)(i * RS * 4));
+        }
+        const int m = m0 + lr;
+        const int n = tn * Cfg::BN + c0 + lc;
+        if (m < geom.M && n < geom.N) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) a[i] *= o.alpha;
+          store_bf16x8(o.out + (long long)n * o.ldo + m, a);
+        }
+      }
+    }
+    cluster_sync();  // the buffers are read before the next round overwrites them (or the CTAs leave)
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, Cfg::ACC_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ epilogues
 
 struct NoRowState {};
 
@@ -790,6 +1119,7 @@ struct EpiStoreBF16 {
   };
   using RowState = NoRowState;
   static constexpr bool kReadsA = false;
+  static constexpr bool kRefillA1 = false;
   static constexpr int kStageOutBytes = 0;
   __device__ static void on_a_stage(const Params&, RowState&, const uint8_t*, bool) {}
   template <int BN>
@@ -825,6 +1155,7 @@ struct EpiPartialF32 {
   };
   using RowState = NoRowState;
   static constexpr bool kReadsA = false;
+  static constexpr bool kRefillA1 = false;
   static constexpr int kStageOutBytes = 0;
   __device__ static void on_a_stage(const Params&, RowState&, const uint8_t*, bool) {}
   template <int BN>
@@ -852,6 +1183,7 @@ struct EpiPartialTMA {
   };
   using RowState = NoRowState;
   static constexpr bool kReadsA = false;
+  static constexpr bool kRefillA1 = false;
   static constexpr int kStageOutBytes = 4 * 2 * 4096;
   __device__ static void on_a_stage(const Params&, RowState&, const uint8_t*, bool) {}
   template <int BN>
