@@ -135,6 +135,27 @@ static ClusterChoice choose_narrow_cluster(int64_t M, int64_t N, int64_t K, bool
   return c;
 }
 
+// The 256 x 256 base GEMMs (forward, dx): the persistent pair kernel (1) or, when
+// its tiles are too few to fill the SM pairs, clusters of 2 or 4 pairs that split
+// K; same time units as above. The persistent kernel overlaps each tile's
+// epilogue with the next tile's main loop, so only its waves count.
+static int choose_wide_cs(int64_t M, int64_t N, int64_t K, int sms) {
+  const int64_t tiles = cdiv(M, 256) * cdiv(N, 256);
+  const int64_t kb = std::max<int64_t>(cdiv(K, 64), 1);
+  const int pairs = std::max(1, sms / 2);
+  double best = (double)cdiv(tiles, pairs) * ((double)kb + 4.0);
+  int cs = 1;
+  for (int c : {2, 4}) {
+    if (kb < 2 * c) break;
+    const double t = (double)cdiv(tiles * c, pairs) * ((double)cdiv(kb, c) + 4.0) + 4.0;
+    if (t < best - 1e-9) {
+      best = t;
+      cs = c;
+    }
+  }
+  return cs;
+}
+
 static NarrowChoice choose_narrow(int64_t M, int64_t N, int64_t K, bool b_mn, int sms) {
   static const int kCandK[] = {64, 128, 256, 384, 512};
   static const int kCandMN[] = {128, 256, 384, 512};
@@ -196,10 +217,18 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
       const ClusterChoice u = choose_narrow_cluster(T, r, d_in, false, p.sms);
       p.u_bn = u.bn;
       p.u_cs = u.cs;
+      p.fwd_cs = choose_wide_cs(T, d_out, cdiv(d_in, 64) * 64 + cdiv(r, 64) * 64, p.sms);
       p.off_su = take((size_t)T * r * 2);
     } else if ((op == DORA_OP_BACKWARD || op == DORA_OP_BACKWARD_FULL) && T > 0) {
       p.off_dz = take((size_t)T * d_out * 2);
-      p.dm_rowblocks = (int)cdiv(T, 256);
+      // Compose backward: 64-column strips x row blocks, sized so that the grid is one
+      // wave at five 256-thread blocks per SM (its register use) and no tail is left.
+      {
+        const int64_t strips = cdiv(d_out, 64), groups = cdiv(T, 32);
+        const int64_t per_strip = std::max<int64_t>(1, (int64_t)p.sms * 5 / strips);
+        p.dm_rows = (int)(32 * cdiv(groups, std::min(per_strip, groups)));
+        p.dm_rowblocks = (int)cdiv(T, p.dm_rows);
+      }
       p.off_dm_part = take((size_t)p.dm_rowblocks * d_out * 4);
       const ClusterChoice du = choose_narrow_cluster(T, r, d_out, true, p.sms);
       p.du_bn = du.bn;
@@ -211,6 +240,7 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
       const ClusterChoice dA = choose_narrow_cluster(d_in, r, T, true, p.sms);
       p.dA_bn = dA.bn;
       p.dA_cs = dA.cs;
+      p.dx_cs = choose_wide_cs(T, d_in, cdiv(d_out, 64) * 64 + cdiv(r, 64) * 64, p.sms);
       // counters of the dm column strips, zeroed by one memset per call
       p.zero_bytes = (size_t)cdiv(d_out, 64) * 4;
       p.off_ctr = take(p.zero_bytes);

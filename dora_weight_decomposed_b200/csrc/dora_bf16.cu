@@ -541,14 +541,13 @@ __global__ void reduce_splits_bf16_kernel(const float* __restrict__ part, int sp
 // Compose backward, one streaming pass over [T x d_out]:
 //   dz[t][i] = g_i * dy[t][i]   (bf16)
 //   part[rb][i] = sum over the row block's t of dy[t][i] * pre[t][i]
-// Block: 256 threads, 64 columns x kCbRows rows. Lane = (row offset 0..3,
-// 8-column vector 0..7), so each warp access covers 4 full 128-byte rows; the
-// per-column sums are combined over the 4 row lanes with shuffles, then over
-// the 8 warps in shared memory. The last row block of a column strip to
-// finish (counter per strip, zero before the launch) sums the strip's
-// partials in row-block order: dm_i = sum / C_i.
-constexpr int kCbRows = 256;
-
+// Block: 256 threads, 64 columns x rows_per_block rows (a multiple of 32; the
+// plan sizes the row blocks so that the whole grid is resident at once). Lane
+// = (row offset 0..3, 8-column vector 0..7), so each warp access covers 4 full
+// 128-byte rows; the per-column sums are combined over the 4 row lanes with
+// shuffles, then over the 8 warps in shared memory. The last row block of a
+// column strip to finish (counter per strip, zero before the launch) sums the
+// strip's partials in row-block order: dm_i = sum / C_i.
 __global__ void __launch_bounds__(256) compose_bwd_bf16_kernel(const __nv_bfloat16* __restrict__ dy,
                                                                const __nv_bfloat16* __restrict__ pre,
                                                                const float* __restrict__ g,
@@ -556,7 +555,8 @@ __global__ void __launch_bounds__(256) compose_bwd_bf16_kernel(const __nv_bfloat
                                                                __nv_bfloat16* __restrict__ dz,
                                                                float* __restrict__ part,
                                                                unsigned int* __restrict__ counters,
-                                                               float* __restrict__ dm, int T, int d_out) {
+                                                               float* __restrict__ dm, int T, int d_out,
+                                                               int rows_per_block) {
   pdl_trigger();
   pdl_wait();
   __shared__ float red[8][64];
@@ -565,8 +565,8 @@ __global__ void __launch_bounds__(256) compose_bwd_bf16_kernel(const __nv_bfloat
   const int cv = lane & 7, ro = lane >> 3;
   const int col = blockIdx.x * 64 + cv * 8;
   const bool col_ok = col < d_out;
-  const int t0 = blockIdx.y * kCbRows;
-  const int t1 = min(T, t0 + kCbRows);
+  const int t0 = blockIdx.y * rows_per_block;
+  const int t1 = min(T, t0 + rows_per_block);
   float acc[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) acc[j] = 0.f;
@@ -713,16 +713,27 @@ static cudaError_t narrow_gemm_1cta(int bn, const GemmArgs& g, float alpha, __nv
   return reduce_splits(part, g.split, sstride, g.M, g.N, alpha, out, ldo, transpose, reduce_name, st);
 }
 
-// Narrow GEMM on CTA-pair clusters (gemm_sm100_pair_cluster_kernel): out =
-// alpha * A B^T in bf16, the K splits of each tile reduced inside its cluster.
+// GEMM on CTA-pair clusters (gemm_sm100_pair_cluster_kernel): the K splits of
+// each 256-row tile reduced inside its cluster; output per ClusterOut.
 template <class Cfg, int CS>
-static cudaError_t launch_pair_cluster(const GemmArgs& g, const NarrowOut& o, cudaStream_t st) {
-  CUtensorMap ta, tb;
+static cudaError_t launch_pair_cluster(const GemmArgs& g, const ClusterOut& o, cudaStream_t st) {
+  CUtensorMap ta0, ta1, tb0, tb1;
+  const int a_box = Cfg::A_MN ? 64 : kBM;
+  const int b_box = Cfg::B_MN ? 64 : Cfg::B_BOX;
   t_detail.clear();
-  if (!make_map(&ta, g.a0, Cfg::A_MN ? 64 : kBM, "A") || !make_map(&tb, g.b0, Cfg::B_MN ? 64 : Cfg::B_BOX, "B"))
+  if (!make_map(&ta0, g.a0, a_box, "A source 0") || !make_map(&tb0, g.b0, b_box, "B source 0"))
     return cudaErrorInvalidValue;
-  const int kb = (int)std::max<int64_t>(ceil_div(g.K0, kBK), 1);
-  GemmGeom geom{g.M, g.N, kb, 0, (int)ceil_div(kb, CS), 0, 0};
+  const int kb0 = (int)ceil_div(g.K0, kBK);
+  const int kb1 = g.K1 > 0 ? (int)ceil_div(g.K1, kBK) : 0;
+  if (kb1 > 0) {
+    if (!make_map(&ta1, g.a1, a_box, "A source 1") || !make_map(&tb1, g.b1, b_box, "B source 1"))
+      return cudaErrorInvalidValue;
+  } else {
+    ta1 = ta0;
+    tb1 = tb0;
+  }
+  const int kb = std::max(kb0 + kb1, 1);
+  GemmGeom geom{g.M, g.N, kb0, kb1, (int)ceil_div(kb, CS), 0, 0};
   const long long tiles = ceil_div(g.N, Cfg::BN) * ceil_div(g.M, 2 * kBM);
   auto kern = gemm_sm100_pair_cluster_kernel<Cfg, CS>;
   constexpr int smem_bytes = PairClusterLayout<Cfg>::SMEM_BYTES;
@@ -748,7 +759,7 @@ static cudaError_t launch_pair_cluster(const GemmArgs& g, const NarrowOut& o, cu
   cfg.numAttrs = 2;
   {
     ProfRange pr(g.name, st);
-    e = cudaLaunchKernelEx(&cfg, kern, ta, tb, geom, o);
+    e = cudaLaunchKernelEx(&cfg, kern, ta0, ta1, tb0, tb1, geom, o);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess)
@@ -757,7 +768,7 @@ static cudaError_t launch_pair_cluster(const GemmArgs& g, const NarrowOut& o, cu
 }
 
 template <int BN, bool A_MN, bool B_MN>
-static cudaError_t pair_cluster_cs(int cs, const GemmArgs& g, const NarrowOut& o, cudaStream_t st) {
+static cudaError_t pair_cluster_cs(int cs, const GemmArgs& g, const ClusterOut& o, cudaStream_t st) {
   using Cfg = PairCfg<BN, A_MN, B_MN>;
   if (cs == 1) return launch_pair_cluster<Cfg, 1>(g, o, st);
   if (cs == 2) return launch_pair_cluster<Cfg, 2>(g, o, st);
@@ -766,10 +777,11 @@ static cudaError_t pair_cluster_cs(int cs, const GemmArgs& g, const NarrowOut& o
   return cudaErrorInvalidValue;
 }
 
+// Narrow GEMM (N = r): out = alpha * A B^T in bf16 on pair clusters.
 template <bool A_MN, bool B_MN>
 static cudaError_t narrow_cluster(int bn, int cs, const GemmArgs& g, float alpha, __nv_bfloat16* out, long long ldo,
                                   bool transpose, cudaStream_t st) {
-  const NarrowOut o{out, ldo, alpha, transpose ? 1 : 0};
+  const ClusterOut o{out, nullptr, nullptr, ldo, alpha, transpose ? 1 : 0, 0};
   if constexpr (!B_MN) {
     if (bn == 64) return pair_cluster_cs<64, A_MN, B_MN>(cs, g, o, st);
   }
@@ -918,6 +930,13 @@ dora_status_t bf16_forward(const dora_desc_t& d, const Plan& p, int64_t T, const
   ba.split.splits = 1;
   ba.name = "fwd_compose_gemm";
   ba.split.kb_per_split = (int)(ceil_div(d_in, kBK) + ceil_div(r, kBK));
+  if (p.fwd_cs > 1) {
+    // Few tiles (small token batches): clusters of pairs split K and compose in the reduction.
+    const ClusterOut o{reinterpret_cast<__nv_bfloat16*>(y), reinterpret_cast<__nv_bfloat16*>(pre_save), gm1, d_out,
+                       1.0f, 0, 1};
+    e = pair_cluster_cs<256, false, false>(p.fwd_cs, ba, o, st);
+    return gemm_status(e, "dora_forward: base GEMM with compose");
+  }
   EpiCompose::Params cp{reinterpret_cast<__nv_bfloat16*>(y), reinterpret_cast<__nv_bfloat16*>(pre_save), gm1,
                         d_out};
   e = launch_gemm_pair<PairCfg<256, false, false>, EpiCompose>(ba, cp, p.sms, st);
@@ -980,7 +999,7 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
       ProfRange pr("compose_bwd", st);
       cudaError_t e = launch_pdl(compose_bwd_bf16_kernel, grid, dim3(256), 0, st,
                                  reinterpret_cast<const __nv_bfloat16*>(dy), reinterpret_cast<const __nv_bfloat16*>(pre),
-                                 g, C, dz, dm_part, ctr, dm, Ti, d_out);
+                                 g, C, dz, dm_part, ctr, dm, Ti, d_out, p.dm_rows);
       if (e != cudaSuccess) return cuda_status(e, "dora_backward: compose backward");
     }
   }
@@ -1036,8 +1055,14 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.split.splits = 1;
     a.name = "dx_gemm";
     a.split.kb_per_split = (int)(ceil_div(d_out, kBK) + ceil_div(r, kBK));
-    EpiStoreBF16::Params sp{reinterpret_cast<__nv_bfloat16*>(dx), d_in, 1.0f, 0};
-    cudaError_t e = launch_gemm_pair<PairCfg<256, false, true>, EpiStoreBF16>(a, sp, p.sms, st);
+    cudaError_t e;
+    if (p.dx_cs > 1) {
+      const ClusterOut o{reinterpret_cast<__nv_bfloat16*>(dx), nullptr, nullptr, d_in, 1.0f, 0, 0};
+      e = pair_cluster_cs<256, false, true>(p.dx_cs, a, o, st);
+    } else {
+      EpiStoreBF16::Params sp{reinterpret_cast<__nv_bfloat16*>(dx), d_in, 1.0f, 0};
+      e = launch_gemm_pair<PairCfg<256, false, true>, EpiStoreBF16>(a, sp, p.sms, st);
+    }
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: dx");
   }
   return DORA_OK;

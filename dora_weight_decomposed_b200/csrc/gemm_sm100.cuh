@@ -839,24 +839,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 
 // ------------------------------------------------------------------ CTA-pair cluster split-K variant
 //
-// For narrow GEMMs (N = the LoRA rank, long K) whose output tiles are too few
-// to fill the GPU: a cluster of 2 * CS CTAs, i.e. CS CTA pairs, computes one
-// 256 x BN output tile, pair z (cluster ranks 2z and 2z + 1) taking the z-th
-// K range. Each pair runs the pair kernels' main loop (its leader is rank 2z;
-// commits go to the pair's two CTAs). The accumulators are then reduced inside
-// the cluster, CW columns at a time: every CTA drains its 128 TMEM rows into
-// its own shared memory (the idle stage ring), and after a cluster barrier
-// CTA (z, q) sums rows [z * 128 / CS, (z + 1) * 128 / CS) of half q over the
-// cluster's CS CTAs of that half, always in split order, by reading their
-// buffers through distributed shared memory, then scales by alpha and stores
-// bf16 (row-major, or transposed out[n][m]). No fp32 partials reach global
-// memory and the result does not depend on timing.
+// For GEMMs whose output tiles are too few to fill the GPU (the narrow rank-r
+// GEMMs with N = r and a long K, and the base GEMMs of small token batches): a
+// cluster of 2 * CS CTAs, i.e. CS CTA pairs, computes one 256 x BN output
+// tile, pair z (cluster ranks 2z and 2z + 1) taking the z-th K range. K may
+// come from two sources back to back, as in the other kernels. Each pair runs
+// the pair kernels' main loop (its leader is rank 2z; commits go to the pair's
+// two CTAs). The accumulators are then reduced inside the cluster, CW columns
+// at a time: every CTA drains its 128 TMEM rows into its own shared memory
+// (the idle stage ring), and after a cluster barrier CTA (z, q) sums rows
+// [z * 128 / CS, (z + 1) * 128 / CS) of half q over the cluster's CS CTAs of
+// that half, always in split order, by reading their buffers through
+// distributed shared memory, and stores them: bf16 alpha * acc (row-major, or
+// transposed out[n][m]), or the forward's compose y = acc + gm1[n] acc with
+// pre = acc. No fp32 partials reach global memory and the result does not
+// depend on timing.
 
-struct NarrowOut {
-  __nv_bfloat16* out;
-  long long ldo;  // row length of out (elements)
+struct ClusterOut {
+  __nv_bfloat16* out;  // alpha * acc, or y in compose mode
+  __nv_bfloat16* pre;  // compose mode: acc rounded (may be null)
+  const float* gm1;    // compose mode: g - 1 per output column
+  long long ldo;       // row length of out (elements)
   float alpha;
-  int transpose;  // 0: out[m][n]; 1: out[n][m]
+  int transpose;       // 0: out[m][n]; 1: out[n][m] (not with compose)
+  int compose;
 };
 
 template <class Cfg>
@@ -888,8 +894,9 @@ __device__ __forceinline__ float4 ld_dsmem_v4(uint32_t cluster_addr) {
 
 template <class Cfg, int CS>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_sm100_pair_cluster_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tB,
-                                   const GemmGeom geom, const NarrowOut o) {
+    gemm_sm100_pair_cluster_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tA1,
+                                   const __grid_constant__ CUtensorMap tB0, const __grid_constant__ CUtensorMap tB1,
+                                   const GemmGeom geom, const ClusterOut o) {
   static_assert(CS == 1 || CS == 2 || CS == 4, "pairs per cluster");
   using L = PairClusterLayout<Cfg>;
   constexpr int STAGES = L::STAGES;
@@ -914,7 +921,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int n_tiles = (geom.N + Cfg::BN - 1) / Cfg::BN;
   const int t = blockIdx.x / (2 * CS);
   const int tm = t / n_tiles, tn = t - tm * n_tiles;
-  const int kb_total = geom.kb0;
+  const int kb_total = geom.kb0 + geom.kb1;
   const int kb_begin = z * geom.kb_per_split;
   const int kb_end = min(kb_total, kb_begin + geom.kb_per_split);
   const int nkb = kb_end > kb_begin ? kb_end - kb_begin : 0;
@@ -930,8 +937,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tA);
-    prefetch_tmap(&tB);
+    prefetch_tmap(&tA0);
+    prefetch_tmap(&tB0);
+    if (geom.kb1 > 0) {
+      prefetch_tmap(&tA1);
+      prefetch_tmap(&tB1);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, Cfg::ACC_COLS);
@@ -957,26 +968,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint8_t* sb = sa + Cfg::A_BYTES;
         const uint32_t fb = mapa_shared(smem_u32(&full[s]), leader);
         if (q == 0) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
-        const int k0 = (kb_begin + i) * kBK;
+        const int kb = kb_begin + i;
+        const bool src1 = kb >= geom.kb0;
+        const int k0 = (src1 ? kb - geom.kb0 : kb) * kBK;
+        const CUtensorMap* ta = src1 ? &tA1 : &tA0;
+        const CUtensorMap* tb = src1 ? &tB1 : &tB0;
         if (!Cfg::A_MN) {
-          tma_load_2d_pair(sa, &tA, fb, k0, m0);
+          tma_load_2d_pair(sa, ta, fb, k0, m0);
         } else {
-          tma_load_2d_pair(sa, &tA, fb, m0, k0);
-          tma_load_2d_pair(sa + 8192, &tA, fb, m0 + 64, k0);
+          tma_load_2d_pair(sa, ta, fb, m0, k0);
+          tma_load_2d_pair(sa + 8192, ta, fb, m0 + 64, k0);
         }
 #pragma unroll
         for (int j = 0; j < Cfg::B0_LOADS; ++j) {
           if (!Cfg::B_MN)
-            tma_load_2d_pair(sb + j * Cfg::B_BOX * 128, &tB, fb, k0, nb0 + j * Cfg::B_BOX);
+            tma_load_2d_pair(sb + j * Cfg::B_BOX * 128, tb, fb, k0, nb0 + j * Cfg::B_BOX);
           else
-            tma_load_2d_pair(sb + j * 8192, &tB, fb, nb0 + j * 64, k0);
+            tma_load_2d_pair(sb + j * 8192, tb, fb, nb0 + j * 64, k0);
         }
 #pragma unroll
         for (int j = 0; j < Cfg::B1_LOADS; ++j) {
           if (!Cfg::B_MN)
-            tma_load_2d_pair(sb + Cfg::B1_OFFSET + j * Cfg::B_BOX * 128, &tB, fb, k0, nb1 + j * Cfg::B_BOX);
+            tma_load_2d_pair(sb + Cfg::B1_OFFSET + j * Cfg::B_BOX * 128, tb, fb, k0, nb1 + j * Cfg::B_BOX);
           else
-            tma_load_2d_pair(sb + Cfg::B1_OFFSET + j * 8192, &tB, fb, nb1 + j * 64, k0);
+            tma_load_2d_pair(sb + Cfg::B1_OFFSET + j * 8192, tb, fb, nb1 + j * 64, k0);
         }
       }
     }
@@ -1066,9 +1081,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int m = m0 + lr;
         const int n = tn * Cfg::BN + c0 + lc;
         if (m < geom.M && n < geom.N) {
+          if (o.compose) {
+            // y = pre + (g - 1) pre in fp32, rounded once; y is not read again in the step.
+            const float4 ga = __ldg(reinterpret_cast<const float4*>(o.gm1 + n));
+            const float4 gb = __ldg(reinterpret_cast<const float4*>(o.gm1 + n + 4));
+            const float gm[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+            float yv[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) a[i] *= o.alpha;
-          store_bf16x8(o.out + (long long)m * o.ldo + n, a);
+            for (int i = 0; i < 8; ++i) yv[i] = fmaf(gm[i], a[i], a[i]);
+            store_bf16x8_cs(o.out + (long long)m * o.ldo + n, yv);
+            if (o.pre) store_bf16x8(o.pre + (long long)m * o.ldo + n, a);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) a[i] *= o.alpha;
+            store_bf16x8(o.out + (long long)m * o.ldo + n, a);
+          }
         }
       }
     } else {
