@@ -106,27 +106,36 @@ static NarrowChoice choose_narrow_1cta(int64_t M, int64_t N, int64_t K, bool b_m
 }
 
 // Tile width and pairs per cluster (K splits reduced in the cluster) of a narrow
-// GEMM on CTA-pair clusters: the narrowest pair tile that covers N, and of 1, 2
-// or 4 pairs per cluster the one with the least estimated time, in units of
-// one k-block's main-loop time: waves of clusters over the SM pairs times the
-// k-blocks of a split, plus a fixed cost per tile (prologue, drain, stores)
-// and per extra cluster round of the reduction. Ties go to fewer splits.
+// GEMM on CTA-pair clusters: the narrowest pair tile that covers N, and of 1 to
+// 4 pairs per cluster the one with the least estimated time, in units of one
+// k-block's main-loop time: waves of clusters (as many at once as the device
+// holds: a cluster must fit in one GPC) times the k-blocks of a split, plus a
+// fixed cost per tile (prologue, pipeline fill, drain, stores) and per extra
+// split of the reduction. Ties go to fewer splits.
 struct ClusterChoice {
   int bn = 128;
   int cs = 1;
 };
+
+// Clusters of cs pairs resident at once: the device's answer, else SMs / (2 cs)
+// less one GPC's worth for clusters above two pairs.
+static int64_t resident_clusters(int cs, int sms) {
+  const int n = max_active_pair_clusters(cs);
+  if (n > 0) return n;
+  const int64_t even = std::max(1, sms / (2 * cs));
+  return cs > 2 ? std::max<int64_t>(1, even - 3) : even;
+}
 
 static ClusterChoice choose_narrow_cluster(int64_t M, int64_t N, int64_t K, bool b_mn, int sms) {
   ClusterChoice c;
   c.bn = b_mn ? (N <= 128 ? 128 : N <= 256 ? 256 : N <= 384 ? 384 : 512) : (int)bn_pair_k(N);
   const int64_t tiles = cdiv(M, 256) * cdiv(N, c.bn);
   const int64_t kb = std::max<int64_t>(cdiv(K, 64), 1);
-  const int pairs = std::max(1, sms / 2);
   double best = 1e300;
-  for (int cs : {1, 2, 4}) {
+  for (int cs : {1, 2, 3, 4}) {
     if (cs > 1 && kb < 2 * cs) break;  // at least two k-blocks per split
-    const int64_t waves = cdiv(tiles * cs, pairs);
-    const double t = (double)waves * ((double)cdiv(kb, cs) + 4.0) + (cs > 1 ? 2.0 * c.bn / 128.0 : 0.0);
+    const int64_t waves = cdiv(tiles, resident_clusters(cs, sms));
+    const double t = (double)waves * ((double)cdiv(kb, cs) + 4.0) + (cs > 1 ? 1.0 * (cs - 1) * c.bn / 128.0 : 0.0);
     if (t < best - 1e-9) {
       best = t;
       c.cs = cs;
@@ -145,9 +154,9 @@ static int choose_wide_cs(int64_t M, int64_t N, int64_t K, int sms) {
   const int pairs = std::max(1, sms / 2);
   double best = (double)cdiv(tiles, pairs) * ((double)kb + 4.0);
   int cs = 1;
-  for (int c : {2, 4}) {
+  for (int c : {2, 3, 4}) {
     if (kb < 2 * c) break;
-    const double t = (double)cdiv(tiles * c, pairs) * ((double)cdiv(kb, c) + 4.0) + 4.0;
+    const double t = (double)cdiv(tiles, resident_clusters(c, sms)) * ((double)cdiv(kb, c) + 4.0) + 2.0 * (c - 1);
     if (t < best - 1e-9) {
       best = t;
       cs = c;

@@ -772,9 +772,78 @@ static cudaError_t pair_cluster_cs(int cs, const GemmArgs& g, const ClusterOut& 
   using Cfg = PairCfg<BN, A_MN, B_MN>;
   if (cs == 1) return launch_pair_cluster<Cfg, 1>(g, o, st);
   if (cs == 2) return launch_pair_cluster<Cfg, 2>(g, o, st);
+  if (cs == 3) return launch_pair_cluster<Cfg, 3>(g, o, st);
   if (cs == 4) return launch_pair_cluster<Cfg, 4>(g, o, st);
   t_detail = "no cluster of " + std::to_string(cs) + " pairs";
   return cudaErrorInvalidValue;
+}
+
+// How many clusters of cs CTA pairs (each CTA one SM: ~200 KB of shared memory)
+// the current device holds at once: a cluster must fit in one GPC, so this is
+// below SMs / (2 cs) for the larger clusters (e.g. 15 clusters of 8 CTAs on a
+// 148-SM B200). Queried once per device and cluster size; 0 if the query fails.
+int max_active_pair_clusters(int cs) {
+  static std::atomic<int> cache[64][5];
+  if (cs < 1 || cs > 4) return 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return 0;
+  }
+  const int hit = cache[dev][cs].load();
+  if (hit != 0) return hit > 0 ? hit : 0;
+  using Cfg = PairCfg<384, false, false>;
+  constexpr int smem_bytes = PairClusterLayout<Cfg>::SMEM_BYTES;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * cs * 64));
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = smem_bytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2 * cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  cudaError_t e = cudaSuccess;
+  switch (cs) {
+    case 1: {
+      static std::atomic<unsigned long long> set{0};
+      auto k = gemm_sm100_pair_cluster_kernel<Cfg, 1>;
+      e = set_smem_once(set, k, smem_bytes);
+      if (e == cudaSuccess) e = cudaOccupancyMaxActiveClusters(&n, k, &cfg);
+      break;
+    }
+    case 2: {
+      static std::atomic<unsigned long long> set{0};
+      auto k = gemm_sm100_pair_cluster_kernel<Cfg, 2>;
+      e = set_smem_once(set, k, smem_bytes);
+      if (e == cudaSuccess) e = cudaOccupancyMaxActiveClusters(&n, k, &cfg);
+      break;
+    }
+    case 3: {
+      static std::atomic<unsigned long long> set{0};
+      auto k = gemm_sm100_pair_cluster_kernel<Cfg, 3>;
+      e = set_smem_once(set, k, smem_bytes);
+      if (e == cudaSuccess) e = cudaOccupancyMaxActiveClusters(&n, k, &cfg);
+      break;
+    }
+    default: {
+      static std::atomic<unsigned long long> set{0};
+      auto k = gemm_sm100_pair_cluster_kernel<Cfg, 4>;
+      e = set_smem_once(set, k, smem_bytes);
+      if (e == cudaSuccess) e = cudaOccupancyMaxActiveClusters(&n, k, &cfg);
+      break;
+    }
+  }
+  if (e != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    cache[dev][cs].store(-1);
+    return 0;
+  }
+  cache[dev][cs].store(n);
+  return n;
 }
 
 // Narrow GEMM (N = r): out = alpha * A B^T in bf16 on pair clusters.

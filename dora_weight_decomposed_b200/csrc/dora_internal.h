@@ -50,6 +50,8 @@ struct Plan {
 inline int bn_pair_k(int64_t r) { return r <= 64 ? 64 : r <= 128 ? 128 : r <= 256 ? 256 : r <= 384 ? 384 : 512; }
 
 int device_sm_count();
+// Clusters of cs CTA pairs (cs = 1..4, one CTA per SM) the current device holds at once; 0 if unknown.
+int max_active_pair_clusters(int cs);
 Plan make_plan(const dora_desc_t& d, int64_t T, int op);
 
 // Thread-local error message for dora_last_error().

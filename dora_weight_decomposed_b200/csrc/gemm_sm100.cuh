@@ -870,39 +870,27 @@ struct PairClusterLayout {
   static constexpr int STAGES_RAW = kSmemBudget / Cfg::STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static_assert(STAGES >= 2, "stages");
-  static constexpr int CW = Cfg::BN < 256 ? Cfg::BN : 256;  // columns reduced per round
-  static constexpr int RS = CW + 4;                         // fp32 row stride of the reduction buffer
+  // Columns reduced per round: the whole tile when its fp32 rows fit the ring, else 256.
+  static constexpr bool ONE_ROUND = 128 * (Cfg::BN + 4) * 4 <= STAGES * Cfg::STAGE_BYTES;
+  static constexpr int CW = ONE_ROUND ? Cfg::BN : 256;
+  static constexpr int RS = CW + 4;  // fp32 row stride of the reduction buffer
   static_assert(Cfg::BN % CW == 0 || Cfg::BN == 384, "whole rounds");
   static_assert(128 * RS * 4 <= STAGES * Cfg::STAGE_BYTES, "reduction buffer fits the ring");
   static constexpr int SMEM_BYTES = STAGES * Cfg::STAGE_BYTES + Cfg::BAR_BYTES + 1024;
 };
-
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t cluster_addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ float4 ld_dsmem_v4(uint32_t cluster_addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(cluster_addr)
-               : "memory");
-  return v;
-}
 
 template <class Cfg, int CS>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_sm100_pair_cluster_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tA1,
                                    const __grid_constant__ CUtensorMap tB0, const __grid_constant__ CUtensorMap tB1,
                                    const GemmGeom geom, const ClusterOut o) {
-  static_assert(CS == 1 || CS == 2 || CS == 4, "pairs per cluster");
+  static_assert(CS >= 1 && CS <= 4, "pairs per cluster");
   using L = PairClusterLayout<Cfg>;
   constexpr int STAGES = L::STAGES;
   constexpr int CW = L::CW;
   constexpr int RS = L::RS;
-  constexpr int ROWS = 128 / CS;  // rows of its half each CTA reduces
+  // Rows of its half each CTA reduces: ROWS (a multiple of 8), the last CTA the rest.
+  constexpr int ROWS = 8 * ((16 + CS - 1) / CS);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
@@ -1036,8 +1024,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     acc_ok = __all_sync(0xffffffffu, mbar_wait(accf, 0));
     tc_fence_after();
   }
-  const uint32_t red_base = smem_u32(red);
-  const int row_lo = z * ROWS;
+  const int row_lo = min(128, z * ROWS);
+  const int rows = min(128, row_lo + ROWS) - row_lo;
 #pragma unroll 1
   for (int c0 = 0; c0 < Cfg::BN; c0 += CW) {
     const int cw = min(CW, Cfg::BN - c0);
@@ -1045,79 +1033,135 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int qq = warp & 3;
       const int row = qq * 32 + lane;
       float* dst = red + row * RS;
+      // 128 columns of TMEM in flight per wait.
 #pragma unroll 1
-      for (int col = 0; col < cw; col += 32) {
-        float v[32];
+      for (int col = 0; col < cw; col += 128) {
+        uint32_t v[4][32];
+        const int nch = min(4, (cw - col) / 32);
         if (nkb > 0 && acc_ok) {
-          tmem_ld32(tmem + ((uint32_t)(qq * 32) << 16) + (uint32_t)(c0 + col), v);
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            if (c < nch) tmem_ld32_async(tmem + ((uint32_t)(qq * 32) << 16) + (uint32_t)(c0 + col + 32 * c), v[c]);
+          tmem_ld_wait();
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = 0.f;
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[c][i] = 0u;
         }
 #pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4*>(dst + col + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        for (int c = 0; c < 4; ++c) {
+          if (c >= nch) break;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(dst + col + 32 * c + i) =
+                make_float4(__uint_as_float(v[c][i]), __uint_as_float(v[c][i + 1]), __uint_as_float(v[c][i + 2]),
+                            __uint_as_float(v[c][i + 3]));
+        }
       }
     }
     tc_fence_before();
     cluster_sync();  // every CTA's round is in its buffer
+    // The CS buffers of this half, read through generic pointers: every load of an item
+    // is issued before the first is summed, and items are summed in split order.
+    const float* srcs[CS];
+#pragma unroll
+    for (int zz = 0; zz < CS; ++zz) srcs[zz] = dsmem_ptr(red, (uint32_t)(2 * zz) + q);
+    // kU items per thread per batch: all their loads are issued before any is summed, so
+    // kU * CS remote reads are in flight at once (each costs several hundred cycles).
+    constexpr int kU = 4;
     if (!o.transpose) {
       // item = (row, 8 columns): out[m][n .. n + 7]
       const int per_row = cw / 8;
-      for (int it = threadIdx.x; it < ROWS * per_row; it += kGemmThreads) {
-        const int lr = row_lo + it / per_row;
-        const int lc = (it % per_row) * 8;
-        const uint32_t off = (uint32_t)((lr * RS + lc) * 4);
-        float a[8];
+      const int n_items = rows * per_row;
+#pragma unroll 1
+      for (int it0 = threadIdx.x; it0 < n_items; it0 += kGemmThreads * kU) {
+        float4 x[kU][CS][2];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) a[i] = 0.f;
+        for (int u = 0; u < kU; ++u) {
+          const int it = it0 + u * kGemmThreads;
+          if (it < n_items) {
+            const int off = (row_lo + it / per_row) * RS + (it % per_row) * 8;
 #pragma unroll
-        for (int zz = 0; zz < CS; ++zz) {
-          const uint32_t src = mapa_shared(red_base + off, (uint32_t)(2 * zz) + q);
-          const float4 x0 = ld_dsmem_v4(src), x1 = ld_dsmem_v4(src + 16);
-          a[0] += x0.x; a[1] += x0.y; a[2] += x0.z; a[3] += x0.w;
-          a[4] += x1.x; a[5] += x1.y; a[6] += x1.z; a[7] += x1.w;
+            for (int zz = 0; zz < CS; ++zz) {
+              x[u][zz][0] = *reinterpret_cast<const float4*>(srcs[zz] + off);
+              x[u][zz][1] = *reinterpret_cast<const float4*>(srcs[zz] + off + 4);
+            }
+          }
         }
-        const int m = m0 + lr;
-        const int n = tn * Cfg::BN + c0 + lc;
-        if (m < geom.M && n < geom.N) {
-          if (o.compose) {
-            // y = pre + (g - 1) pre in fp32, rounded once; y is not read again in the step.
-            const float4 ga = __ldg(reinterpret_cast<const float4*>(o.gm1 + n));
-            const float4 gb = __ldg(reinterpret_cast<const float4*>(o.gm1 + n + 4));
-            const float gm[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-            float yv[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) yv[i] = fmaf(gm[i], a[i], a[i]);
-            store_bf16x8_cs(o.out + (long long)m * o.ldo + n, yv);
-            if (o.pre) store_bf16x8(o.pre + (long long)m * o.ldo + n, a);
-          } else {
+        for (int u = 0; u < kU; ++u) {
+          const int it = it0 + u * kGemmThreads;
+          if (it >= n_items) break;
+          const int lr = row_lo + it / per_row;
+          const int lc = (it % per_row) * 8;
+          float a[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) a[i] *= o.alpha;
-            store_bf16x8(o.out + (long long)m * o.ldo + n, a);
+          for (int i = 0; i < 8; ++i) a[i] = 0.f;
+#pragma unroll
+          for (int zz = 0; zz < CS; ++zz) {
+            a[0] += x[u][zz][0].x; a[1] += x[u][zz][0].y; a[2] += x[u][zz][0].z; a[3] += x[u][zz][0].w;
+            a[4] += x[u][zz][1].x; a[5] += x[u][zz][1].y; a[6] += x[u][zz][1].z; a[7] += x[u][zz][1].w;
+          }
+          const int m = m0 + lr;
+          const int n = tn * Cfg::BN + c0 + lc;
+          if (m < geom.M && n < geom.N) {
+            if (o.compose) {
+              // y = pre + (g - 1) pre in fp32, rounded once; y is not read again in the step.
+              const float4 ga = __ldg(reinterpret_cast<const float4*>(o.gm1 + n));
+              const float4 gb = __ldg(reinterpret_cast<const float4*>(o.gm1 + n + 4));
+              const float gm[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+              float yv[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) yv[i] = fmaf(gm[i], a[i], a[i]);
+              store_bf16x8_cs(o.out + (long long)m * o.ldo + n, yv);
+              if (o.pre) store_bf16x8(o.pre + (long long)m * o.ldo + n, a);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) a[i] *= o.alpha;
+              store_bf16x8(o.out + (long long)m * o.ldo + n, a);
+            }
           }
         }
       }
     } else {
       // item = (column, 8 rows): out[n][m .. m + 7]
-      for (int it = threadIdx.x; it < (ROWS / 8) * cw; it += kGemmThreads) {
-        const int lc = it % cw;
-        const int lr = row_lo + (it / cw) * 8;
-        float a[8];
+      const int n_items = (rows / 8) * cw;
+#pragma unroll 1
+      for (int it0 = threadIdx.x; it0 < n_items; it0 += kGemmThreads * kU) {
+        float x[kU][CS][8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) a[i] = 0.f;
+        for (int u = 0; u < kU; ++u) {
+          const int it = it0 + u * kGemmThreads;
+          if (it < n_items) {
+            const int lc = it % cw;
+            const int lr = row_lo + (it / cw) * 8;
 #pragma unroll
-        for (int zz = 0; zz < CS; ++zz) {
-          const uint32_t src = mapa_shared(red_base + (uint32_t)((lr * RS + lc) * 4), (uint32_t)(2 * zz) + q);
+            for (int zz = 0; zz < CS; ++zz)
 #pragma unroll
-          for (int i = 0; i < 8; ++i) a[i] += ld_dsmem_f32(src + (uint32_t)(i * RS * 4));
+              for (int i = 0; i < 8; ++i) x[u][zz][i] = srcs[zz][(lr + i) * RS + lc];
+          }
         }
-        const int m = m0 + lr;
-        const int n = tn * Cfg::BN + c0 + lc;
-        if (m < geom.M && n < geom.N) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) a[i] *= o.alpha;
-          store_bf16x8(o.out + (long long)n * o.ldo + m, a);
+        for (int u = 0; u < kU; ++u) {
+          const int it = it0 + u * kGemmThreads;
+          if (it >= n_items) break;
+          const int lc = it % cw;
+          const int lr = row_lo + (it / cw) * 8;
+          float a[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) a[i] = 0.f;
+#pragma unroll
+          for (int zz = 0; zz < CS; ++zz)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) a[i] += x[u][zz][i];
+          const int m = m0 + lr;
+          const int n = tn * Cfg::BN + c0 + lc;
+          if (m < geom.M && n < geom.N) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) a[i] *= o.alpha;
+            store_bf16x8(o.out + (long long)n * o.ldo + m, a);
+          }
         }
       }
     }

@@ -34,6 +34,7 @@ constexpr int kGramOpBytes = kGramTile * 64 * 2;      // one 128-row x 64-column
 constexpr int kGramStageBytes = 2 * kGramOpBytes;
 constexpr int kGramRedLd = kGramTile + 4;             // fp32 row stride of the reduction buffer (floats)
 constexpr int kGramSmemBytes = kGramStages * kGramStageBytes + 256 + 1024;
+constexpr int kGramTrOffset = 128 * 1024;             // transposed bf16 staging (after the fp32 buffer)
 static_assert(kGramTile * kGramRedLd * 4 <= kGramStages * kGramStageBytes, "reduction buffer fits the ring");
 
 struct GramParams {
@@ -57,15 +58,6 @@ __device__ __forceinline__ void gram_tile(int t, int nt, int& ti, int& tj) {
     ++ti;
   }
   tj = ti + (t - first);
-}
-
-__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t cluster_addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(cluster_addr)
-               : "memory");
-  return v;
 }
 
 template <int CS>
@@ -172,35 +164,56 @@ __global__ void __launch_bounds__(192, 1) gram_cluster_kernel(const __grid_const
   tc_fence_before();
   cluster_sync();  // every CTA's buffer is complete and visible to the cluster
 
-  // Rows [crank * kRows, +kRows) of the tile: the cluster's slices summed in rank order.
+  // Rows [crank * kRows, +kRows) of the tile: the cluster's slices summed in rank order,
+  // read through generic pointers so that all CS loads of an item are in flight at once.
   constexpr int kRows = kGramTile / CS;
-  const uint32_t red_base = smem_u32(red);
+  const float* srcs[CS];
+#pragma unroll
+  for (int z = 0; z < CS; ++z) srcs[z] = dsmem_ptr(red, (uint32_t)z);
   const int two_rp = 2 * p.rp;
+  // Staging of the transposed tile (after the fp32 buffer in the idle ring).
+  constexpr int kTrLd = kRows + 8;  // bf16 row stride, 16-byte aligned
+  __nv_bfloat16* tr_hi = reinterpret_cast<__nv_bfloat16*>(smem + kGramTrOffset);
+  __nv_bfloat16* tr_lo = tr_hi + kGramTile * kTrLd;
+  static_assert(kGramTile * kGramRedLd * 4 <= kGramTrOffset &&
+                    kGramTrOffset + 2 * kGramTile * kTrLd * 2 <= kGramStages * kGramStageBytes,
+                "transposed staging fits the ring after the fp32 buffer");
   for (int idx = threadIdx.x; idx < kRows * (kGramTile / 4); idx += blockDim.x) {
     const int lr = (int)crank * kRows + idx / (kGramTile / 4);
     const int lc = (idx % (kGramTile / 4)) * 4;
-    const uint32_t off = (uint32_t)((lr * kGramRedLd + lc) * 4);
+    const int off = lr * kGramRedLd + lc;
+    float4 v[CS];
+#pragma unroll
+    for (int z = 0; z < CS; ++z) v[z] = *reinterpret_cast<const float4*>(srcs[z] + off);
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int z = 0; z < CS; ++z) {
-      const float4 v = ld_dsmem_f4(mapa_shared(red_base + off, (uint32_t)z));
-      a.x += v.x;
-      a.y += v.y;
-      a.z += v.z;
-      a.w += v.w;
+      a.x += v[z].x;
+      a.y += v[z].y;
+      a.z += v[z].z;
+      a.w += v[z].w;
     }
     const float xs[4] = {p.scale * a.x, p.scale * a.y, p.scale * a.z, p.scale * a.w};
     const int gi = ti * kGramTile + lr;
     const int gj = tj * kGramTile + lc;
-    if (gi >= p.r) continue;
     __nv_bfloat16 hi[4], lo[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const bool valid = gj + j < p.r;  // columns r .. rp - 1 are zero padding
+      const bool valid = gi < p.r && gj + j < p.r;  // outside r: zero (the padding of gs2)
       const __nv_bfloat16 h = __float2bfloat16_rn(valid ? xs[j] : 0.f);
       hi[j] = h;
       lo[j] = __float2bfloat16_rn(valid ? xs[j] - __bfloat162float(h) : 0.f);
     }
+    if (!diag) {
+      // The transposed values, staged so that tile (tj, ti) is written in whole rows below.
+      const int lrl = lr - (int)crank * kRows;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        tr_hi[(lc + j) * kTrLd + lrl] = hi[j];
+        tr_lo[(lc + j) * kTrLd + lrl] = lo[j];
+      }
+    }
+    if (gi >= p.r) continue;
     __nv_bfloat16* rowp = p.gs2 + (size_t)gi * two_rp;
     if (gj + 3 < p.rp) {
       *reinterpret_cast<uint2*>(rowp + gj) = *reinterpret_cast<const uint2*>(hi);
@@ -213,15 +226,23 @@ __global__ void __launch_bounds__(192, 1) gram_cluster_kernel(const __grid_const
           rowp[p.rp + gj + j] = lo[j];
         }
     }
-    if (!diag) {
-      // G is symmetric: the same values at (gj + j, gi).
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (gj + j < p.r) {
-          __nv_bfloat16* t = p.gs2 + (size_t)(gj + j) * two_rp;
-          t[gi] = hi[j];
-          t[p.rp + gi] = lo[j];
-        }
+  }
+  if (!diag) {
+    // G is symmetric: rows tj * 128 + c of gs2 receive this CTA's kRows columns
+    // ti * 128 + crank * kRows .. as contiguous 16-byte pieces (hi, then lo).
+    __syncthreads();
+    const int gi0 = ti * kGramTile + (int)crank * kRows;
+    constexpr int kPieces = kRows / 8;
+    for (int idx = threadIdx.x; idx < kGramTile * kPieces * 2; idx += blockDim.x) {
+      const int half = idx / (kGramTile * kPieces);
+      const int rem = idx - half * kGramTile * kPieces;
+      const int c = rem / kPieces;
+      const int pc = (rem - c * kPieces) * 8;
+      const int R = tj * kGramTile + c;
+      if (R >= p.r || gi0 + pc >= p.rp) continue;
+      const __nv_bfloat16* src = (half ? tr_lo : tr_hi) + c * kTrLd + pc;
+      *reinterpret_cast<uint4*>(p.gs2 + (size_t)R * two_rp + (half ? p.rp : 0) + gi0 + pc) =
+          *reinterpret_cast<const uint4*>(src);
     }
   }
   cluster_sync();  // no CTA leaves while another still reads its buffer

@@ -237,6 +237,17 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
   return out;
 }
 
+// Generic address of the same shared-memory location in CTA `rank` of the
+// cluster. Loads through it are ordinary loads, so the compiler can keep
+// several in flight (a distributed shared memory read costs hundreds of
+// cycles); the cluster barriers around them order them.
+template <class T>
+__device__ __forceinline__ const T* dsmem_ptr(const T* p, uint32_t rank) {
+  uint64_t out;
+  asm("mapa.u64 %0, %1, %2;" : "=l"(out) : "l"(reinterpret_cast<uint64_t>(p)), "r"(rank));
+  return reinterpret_cast<const T*>(out);
+}
+
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }

@@ -37,10 +37,17 @@ SMALL = {
     "r8_one_token": ("c2", dict(d_out=8, d_in=8, r=8, T=1)),
     "r16_wide": ("c2", dict(d_out=640, d_in=384, r=16, T=200)),
     "r64_near_unity": ("c4a", dict(d_out=384, d_in=1024, T=130)),
-    # 28 row tiles x 2 K splits leave 36 SMs beside the norm GEMM: the Gram takes 4 CTAs per tile;
-    # the forward GEMM splits K over clusters of 2 pairs, dx over 4.
-    "gram_beside_norm": ("c3", dict(d_out=7168, d_in=2048, T=64)),
 }
+
+
+def test_gram_beside_norm_parity():
+    """28 row tiles x 2 K splits leave 36 SMs beside the norm GEMM: the Gram takes 4 CTAs per
+    tile and runs while the norm GEMM streams W0; the forward GEMM splits K over clusters of 2
+    pairs and dx over 4."""
+    wl = workload("c3", d_out=7168, d_in=2048, T=64)
+    inp = tl.prepare(wl)
+    out = tl.run_gpu(tl.to_device(inp), wl.s)
+    tl.check_all(out, tl.run_oracle(inp), inp, what="gram beside norm")
 
 
 @pytest.mark.parametrize("name", sorted(SMALL))
