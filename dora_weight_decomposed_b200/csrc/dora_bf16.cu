@@ -97,7 +97,8 @@ static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  // Under the kernel profiler each launch is timed on its own: no early start.
+  attr[0].val.programmaticStreamSerializationAllowed = profiling_on() ? 0 : 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
@@ -320,9 +321,16 @@ struct EpiNorm {
     const bool row_ok = c.m < g.M;
     mbar_wait(c.aux_bar, 0);
     const int t = c.row & 7;
+    // This thread's row in each 64-column slab of the prefetched B rows.
+    constexpr int kSlabs = (BN + 63) / 64;
     const int sps = c.stage_stride / 16384;
-    float dot = 0.f;
-#pragma unroll 1
+    const uint8_t* slab_row[kSlabs];
+#pragma unroll
+    for (int sl = 0; sl < kSlabs; ++sl)
+      slab_row[sl] = c.stage_smem + ((c.refill_first + sl / sps) % c.ring_stages) * c.stage_stride +
+                     (sl % sps) * 16384 + c.row * 128;
+    float dot8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // eight independent FMA chains
+#pragma unroll
     for (int col0 = 0; col0 < BN; col0 += 128) {
       constexpr int kMaxChunks = BN < 128 ? BN / 32 : 4;
       uint32_t v[kMaxChunks][32];
@@ -346,17 +354,16 @@ struct EpiNorm {
           const int n = col0 + 32 * q + 8 * j;
           if (n < p.r) {
             const int slab = n >> 6, chunk = (n & 63) >> 3;
-            const uint8_t* base = c.stage_smem + ((c.refill_first + slab / sps) % c.ring_stages) * c.stage_stride +
-                                  (slab % sps) * 16384;
-            const uint4 w = *reinterpret_cast<const uint4*>(base + c.row * 128 + ((chunk ^ t) << 4));
+            const uint4 w = *reinterpret_cast<const uint4*>(slab_row[slab] + ((chunk ^ t) << 4));
             float b[8];
             unpack_bf16x8(w, b);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) dot = fmaf(b[i], __uint_as_float(v[q][8 * j + i]), dot);
+            for (int i = 0; i < 8; ++i) dot8[i] = fmaf(b[i], __uint_as_float(v[q][8 * j + i]), dot8[i]);
           }
         }
       }
     }
+    const float dot = ((dot8[0] + dot8[1]) + (dot8[2] + dot8[3])) + ((dot8[4] + dot8[5]) + (dot8[6] + dot8[7]));
     const float part = fmaf(p.two_s, dot, st.ss);
     if (c.splits == 1) {
       if (row_ok) finish(p, c.m, part);
@@ -750,7 +757,8 @@ static cudaError_t launch_pair_cluster(const GemmArgs& g, const ClusterOut& o, c
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  // Under the kernel profiler each launch is timed on its own: no early start.
+  attr[0].val.programmaticStreamSerializationAllowed = profiling_on() ? 0 : 1;
   attr[1].id = cudaLaunchAttributeClusterDimension;
   attr[1].val.clusterDim.x = 2 * CS;
   attr[1].val.clusterDim.y = 1;
@@ -888,7 +896,8 @@ static cudaError_t launch_gram_cs(const CUtensorMap& ta, const GramParams& gp0, 
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  // Under the kernel profiler each launch is timed on its own: no early start.
+  attr[0].val.programmaticStreamSerializationAllowed = profiling_on() ? 0 : 1;
   attr[1].id = cudaLaunchAttributeClusterDimension;
   attr[1].val.clusterDim.x = CS;
   attr[1].val.clusterDim.y = 1;

@@ -103,6 +103,11 @@ dora_status_t vera_compose(const dora_desc_t& d, const void* Bs, const float* b,
 dora_status_t vera_grad(const dora_desc_t& d, const Plan& p, const void* Bs, const float* b, const float* dv,
                         const void* dBp, float* db, float* dd, uint8_t* ws, cudaStream_t st);
 
+// True while the kernel profiler is on (dora_profile_start .. dora_profile_stop):
+// launches then drop programmatic dependent launch, so that the events around
+// each kernel time that kernel alone.
+bool profiling_on();
+
 // Brackets one kernel launch with profiling events when profiling is on.
 class ProfRange {
  public:

@@ -1,6 +1,7 @@
 // Kernel-level timing inside the library. When started, every kernel the
 // library launches is bracketed by a pair of CUDA events recorded on the
-// launch stream; during stream capture the events become event-record nodes of
+// launch stream, and launched without programmatic dependent launch (so that
+// it cannot start under its predecessor's events); during stream capture the events become event-record nodes of
 // the graph, so each replay of the graph re-times the same kernels. Reading
 // waits for the events and reports each launch's duration. Meant for
 // benchmarks on one host thread; off by default and free when off.
@@ -43,6 +44,12 @@ cudaError_t record(cudaEvent_t ev, cudaStream_t st) {
 }
 
 }  // namespace
+
+bool profiling_on() {
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> lk(p.mu);
+  return p.on;
+}
 
 ProfRange::ProfRange(const char* name, cudaStream_t st) : st_(st), idx_(-1) {
   Profiler& p = prof();

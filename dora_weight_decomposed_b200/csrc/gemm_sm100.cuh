@@ -1296,17 +1296,20 @@ struct EpiPartialTMA {
 // completes the count re-reads all partials in split order (so the result does
 // not depend on which CTA came last). Called by all 128 epilogue threads after
 // their partial stores; true in the CTA that completes the tile.
+// Ordering: the barrier orders every epilogue thread's partial stores before
+// thread 0's counter update, which releases them at GPU scope (release is
+// cumulative over what the barrier ordered before it); in the completing CTA
+// the same acq_rel update acquires the other CTAs' released stores, and the
+// second barrier passes that on to the threads that read them.
 __device__ __forceinline__ bool split_arrive_last(const EpiCtx& c, unsigned int* counters) {
-  __threadfence();
   asm volatile("bar.sync 1, 128;" ::: "memory");
   if (c.row == 0) {
-    const unsigned int old = atomicAdd(&counters[c.tile_id], 1u);
+    unsigned int old;
+    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(old) : "l"(counters + c.tile_id) : "memory");
     *c.flag = (old == (unsigned int)(c.splits - 1)) ? 1u : 0u;
   }
   asm volatile("bar.sync 1, 128;" ::: "memory");
-  const bool last = *reinterpret_cast<volatile uint32_t*>(c.flag) != 0u;
-  if (last) __threadfence();
-  return last;
+  return *reinterpret_cast<volatile uint32_t*>(c.flag) != 0u;
 }
 
 }  // namespace dora

@@ -178,53 +178,67 @@ __global__ void __launch_bounds__(192, 1) gram_cluster_kernel(const __grid_const
   static_assert(kGramTile * kGramRedLd * 4 <= kGramTrOffset &&
                     kGramTrOffset + 2 * kGramTile * kTrLd * 2 <= kGramStages * kGramStageBytes,
                 "transposed staging fits the ring after the fp32 buffer");
-  for (int idx = threadIdx.x; idx < kRows * (kGramTile / 4); idx += blockDim.x) {
-    const int lr = (int)crank * kRows + idx / (kGramTile / 4);
-    const int lc = (idx % (kGramTile / 4)) * 4;
-    const int off = lr * kGramRedLd + lc;
-    float4 v[CS];
+  // Four items per thread per batch: all their remote loads are issued before any is summed.
+  constexpr int kItems = kRows * (kGramTile / 4);
+  constexpr int kU = 4;
+  for (int idx0 = threadIdx.x; idx0 < kItems; idx0 += 192 * kU) {
+    float4 vv[kU][CS];
 #pragma unroll
-    for (int z = 0; z < CS; ++z) v[z] = *reinterpret_cast<const float4*>(srcs[z] + off);
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < kU; ++u) {
+      const int idx = idx0 + u * 192;
+      if (idx < kItems) {
+        const int off = ((int)crank * kRows + idx / (kGramTile / 4)) * kGramRedLd + (idx % (kGramTile / 4)) * 4;
 #pragma unroll
-    for (int z = 0; z < CS; ++z) {
-      a.x += v[z].x;
-      a.y += v[z].y;
-      a.z += v[z].z;
-      a.w += v[z].w;
-    }
-    const float xs[4] = {p.scale * a.x, p.scale * a.y, p.scale * a.z, p.scale * a.w};
-    const int gi = ti * kGramTile + lr;
-    const int gj = tj * kGramTile + lc;
-    __nv_bfloat16 hi[4], lo[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const bool valid = gi < p.r && gj + j < p.r;  // outside r: zero (the padding of gs2)
-      const __nv_bfloat16 h = __float2bfloat16_rn(valid ? xs[j] : 0.f);
-      hi[j] = h;
-      lo[j] = __float2bfloat16_rn(valid ? xs[j] - __bfloat162float(h) : 0.f);
-    }
-    if (!diag) {
-      // The transposed values, staged so that tile (tj, ti) is written in whole rows below.
-      const int lrl = lr - (int)crank * kRows;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        tr_hi[(lc + j) * kTrLd + lrl] = hi[j];
-        tr_lo[(lc + j) * kTrLd + lrl] = lo[j];
+        for (int z = 0; z < CS; ++z) vv[u][z] = *reinterpret_cast<const float4*>(srcs[z] + off);
       }
     }
-    if (gi >= p.r) continue;
-    __nv_bfloat16* rowp = p.gs2 + (size_t)gi * two_rp;
-    if (gj + 3 < p.rp) {
-      *reinterpret_cast<uint2*>(rowp + gj) = *reinterpret_cast<const uint2*>(hi);
-      *reinterpret_cast<uint2*>(rowp + p.rp + gj) = *reinterpret_cast<const uint2*>(lo);
-    } else {
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (gj + j < p.rp) {
-          rowp[gj + j] = hi[j];
-          rowp[p.rp + gj + j] = lo[j];
+    for (int u = 0; u < kU; ++u) {
+      const int idx = idx0 + u * 192;
+      if (idx >= kItems) break;
+      const int lr = (int)crank * kRows + idx / (kGramTile / 4);
+      const int lc = (idx % (kGramTile / 4)) * 4;
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int z = 0; z < CS; ++z) {
+        a.x += vv[u][z].x;
+        a.y += vv[u][z].y;
+        a.z += vv[u][z].z;
+        a.w += vv[u][z].w;
+      }
+      const float xs[4] = {p.scale * a.x, p.scale * a.y, p.scale * a.z, p.scale * a.w};
+      const int gi = ti * kGramTile + lr;
+      const int gj = tj * kGramTile + lc;
+      __nv_bfloat16 hi[4], lo[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const bool valid = gi < p.r && gj + j < p.r;  // outside r: zero (the padding of gs2)
+        const __nv_bfloat16 h = __float2bfloat16_rn(valid ? xs[j] : 0.f);
+        hi[j] = h;
+        lo[j] = __float2bfloat16_rn(valid ? xs[j] - __bfloat162float(h) : 0.f);
+      }
+      if (!diag) {
+        // The transposed values, staged so that tile (tj, ti) is written in whole rows below.
+        const int lrl = lr - (int)crank * kRows;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          tr_hi[(lc + j) * kTrLd + lrl] = hi[j];
+          tr_lo[(lc + j) * kTrLd + lrl] = lo[j];
         }
+      }
+      if (gi >= p.r) continue;  // (the next item of the batch)
+      __nv_bfloat16* rowp = p.gs2 + (size_t)gi * two_rp;
+      if (gj + 3 < p.rp) {
+        *reinterpret_cast<uint2*>(rowp + gj) = *reinterpret_cast<const uint2*>(hi);
+        *reinterpret_cast<uint2*>(rowp + p.rp + gj) = *reinterpret_cast<const uint2*>(lo);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (gj + j < p.rp) {
+            rowp[gj + j] = hi[j];
+            rowp[p.rp + gj + j] = lo[j];
+          }
+      }
     }
   }
   if (!diag) {
