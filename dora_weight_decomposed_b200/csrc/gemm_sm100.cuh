@@ -1066,7 +1066,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // is issued before the first is summed, and items are summed in split order.
     const float* srcs[CS];
 #pragma unroll
-    for (int zz = 0; zz < CS; ++zz) srcs[zz] = dsmem_ptr(red, (uint32_t)(2 * zz) + q);
+    for (int zz = 0; zz < CS; ++zz) srcs[zz] = zz == z ? red : dsmem_ptr(red, (uint32_t)(2 * zz) + q);  // own: local
     // kU items per thread per batch: all their loads are issued before any is summed, so
     // kU * CS remote reads are in flight at once (each costs several hundred cycles).
     constexpr int kU = 4;

@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(192, 1) gram_cluster_kernel(const __grid_const
   constexpr int kRows = kGramTile / CS;
   const float* srcs[CS];
 #pragma unroll
-  for (int z = 0; z < CS; ++z) srcs[z] = dsmem_ptr(red, (uint32_t)z);
+  for (int z = 0; z < CS; ++z) srcs[z] = z == (int)crank ? red : dsmem_ptr(red, (uint32_t)z);  // own: local
   const int two_rp = 2 * p.rp;
   // Staging of the transposed tile (after the fp32 buffer in the idle ring).
   constexpr int kTrLd = kRows + 8;  // bf16 row stride, 16-byte aligned
