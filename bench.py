@@ -752,7 +752,15 @@ def _table(args):
         print(json.dumps(sig(line)), flush=True)
         rows.append((key, wl, line))
         torch.cuda.empty_cache()
-    out = ["| workload | dtype | tokens/s | µs per step | norm / forward / backward µs | layer roofline µs "
+    out = ["# Layer step per workload, one B200",
+           "",
+           f"`python bench.py --table {os.path.basename(args.table)} --steps {args.steps} --warmup {args.warmup}`: "
+           "per workload the layer step (dora_norm + dora_forward + dora_backward, one CUDA graph per call, "
+           "L2 flushed before every timed step, CUDA events on the launching stream), synthetic inputs of "
+           "the workload's shapes. The layer roofline is the slower of flops / measured burst bf16 peak and "
+           "bytes / measured HBM copy rate per call.",
+           "",
+           "| workload | dtype | tokens/s | µs per step | norm / forward / backward µs | layer roofline µs "
            "(tokens/s) | fraction of roofline | norm TFLOP/s | launches per step |",
            "|---|---|---|---|---|---|---|---|---|"]
     for key, wl, l in rows:
