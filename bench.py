@@ -95,6 +95,7 @@ def kernel_work(name, wl):
         "du_gemm": (2 * T * do * r, b * (T * do + do * r + T * r)),
         "dB_gemm": (2 * T * do * r, b * (T * do + T * r + do * r)),
         "dA_gemm": (2 * T * di * r, b * (T * di + T * r + r * di)),
+        "dBA_gemm": (2 * T * r * (do + di), b * (T * do + T * r + do * r + T * di + T * r + r * di)),
         "dx_gemm": (2 * T * di * (do + r), b * (T * do + do * di + T * r + r * di + T * di)),
         "merge_gemm": (2 * do * di * r + 3 * do * di, b * (2 * do * di + do * r + r * di) + 4 * do),
     }

@@ -165,6 +165,28 @@ static int choose_wide_cs(int64_t M, int64_t N, int64_t K, int sms) {
   return cs;
 }
 
+// dB and dA (both K = T, tile width bn) in one grouped persistent launch of whole
+// tiles, or as two cluster split-K launches: estimated microseconds at ~1.9 GHz,
+// a pair k-block taking the longer of its MMAs and its operand loads (~110 GB/s
+// per SM); a fixed 4 us for the grouped launch and 10 us per cluster launch
+// (prologue, accumulator drain, cluster reduction, stores).
+static bool dBA_grouped(int64_t d_out, int64_t d_in, int64_t r, int64_t T, int bn, int sms) {
+  const int64_t kb = std::max<int64_t>(cdiv(T, 64), 1);
+  const int pairs = std::max(1, sms / 2);
+  const double kb_us = std::max(2.0 * 256.0 * bn * 64.0 / 23.0e6, (16384.0 + 64.0 * bn) / 110.0e3);
+  const int64_t tB = cdiv(d_out, 256) * cdiv(r, bn), tA = cdiv(d_in, 256) * cdiv(r, bn);
+  const double grouped = (double)cdiv(tB + tA, pairs) * (double)kb * kb_us + 4.0;
+  auto clustered = [&](int64_t tiles) {
+    double best = 1e300;
+    for (int cs : {1, 2, 3, 4}) {
+      if (cs > 1 && kb < 2 * cs) break;
+      best = std::min(best, (double)cdiv(tiles, resident_clusters(cs, sms)) * (double)cdiv(kb, cs) * kb_us + 10.0);
+    }
+    return best;
+  };
+  return grouped <= clustered(tB) + clustered(tA);
+}
+
 static NarrowChoice choose_narrow(int64_t M, int64_t N, int64_t K, bool b_mn, int sms) {
   static const int kCandK[] = {64, 128, 256, 384, 512};
   static const int kCandMN[] = {128, 256, 384, 512};
@@ -249,6 +271,7 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
       const ClusterChoice dA = choose_narrow_cluster(d_in, r, T, true, p.sms);
       p.dA_bn = dA.bn;
       p.dA_cs = dA.cs;
+      p.dBA_grouped = dBA_grouped(d_out, d_in, r, T, p.dB_bn, p.sms) ? 1 : 0;
       p.dx_cs = choose_wide_cs(T, d_in, cdiv(d_out, 64) * 64 + cdiv(r, 64) * 64, p.sms);
       // counters of the dm column strips, zeroed by one memset per call
       p.zero_bytes = (size_t)cdiv(d_out, 64) * 4;

@@ -25,6 +25,7 @@
 #include "dora_internal.h"
 #include "gemm_sm100.cuh"
 #include "gram_sm100.cuh"
+#include "grouped_sm100.cuh"
 #include "merge_sm100.cuh"
 
 namespace dora {
@@ -870,6 +871,88 @@ static cudaError_t narrow_cluster(int bn, int cs, const GemmArgs& g, float alpha
   return cudaErrorInvalidValue;
 }
 
+// ============================================================== grouped launches
+
+// One or two GEMMs with the same K sources and tile shape in one persistent
+// launch (gemm_sm100_pair_grouped_kernel): whole tiles, at most `pairs` CTA pairs.
+template <class Cfg>
+static cudaError_t launch_grouped(const GemmArgs* gs, const ClusterOut* os, int nprob, int pairs, const char* name,
+                                  cudaStream_t st) {
+  GroupMaps maps{};
+  GroupGeom geom{};
+  const int a_box = Cfg::A_MN ? 64 : kBM;
+  const int b_box = Cfg::B_MN ? 64 : Cfg::B_BOX;
+  t_detail.clear();
+  int tiles = 0;
+  for (int j = 0; j < nprob; ++j) {
+    const GemmArgs& g = gs[j];
+    const int kb0 = (int)ceil_div(g.K0, kBK);
+    const int kb1 = g.K1 > 0 ? (int)ceil_div(g.K1, kBK) : 0;
+    if ((j > 0 && (kb0 != geom.kb0 || kb1 != geom.kb1)) || os[j].compose) {
+      t_detail = "grouped problems need the same K and a plain output";
+      return cudaErrorInvalidValue;
+    }
+    geom.kb0 = kb0;
+    geom.kb1 = kb1;
+    if (!make_map(&maps.a0[j], g.a0, a_box, "A source 0") || !make_map(&maps.b0[j], g.b0, b_box, "B source 0"))
+      return cudaErrorInvalidValue;
+    if (kb1 > 0) {
+      if (!make_map(&maps.a1[j], g.a1, a_box, "A source 1") || !make_map(&maps.b1[j], g.b1, b_box, "B source 1"))
+        return cudaErrorInvalidValue;
+    } else {
+      maps.a1[j] = maps.a0[j];
+      maps.b1[j] = maps.b0[j];
+    }
+    GroupProblem& pr = geom.pr[j];
+    pr.M = g.M;
+    pr.N = g.N;
+    pr.n_tiles = (int)ceil_div(g.N, Cfg::BN);
+    pr.tile_base = tiles;
+    pr.o = os[j];
+    tiles += (int)(ceil_div(g.M, 2 * kBM) * pr.n_tiles);
+  }
+  for (int j = nprob; j < 2; ++j) {
+    maps.a0[j] = maps.a0[0];
+    maps.a1[j] = maps.a1[0];
+    maps.b0[j] = maps.b0[0];
+    maps.b1[j] = maps.b1[0];
+    geom.pr[j] = geom.pr[0];
+    geom.pr[j].tile_base = tiles;
+  }
+  geom.tiles = tiles;
+  geom.nprob = nprob;
+  const int P = std::max(1, std::min(pairs, tiles));
+  auto kern = gemm_sm100_pair_grouped_kernel<Cfg>;
+  constexpr int smem_bytes = GroupLayout<Cfg>::SMEM_BYTES;
+  static std::atomic<unsigned long long> smem_set{0};
+  cudaError_t e = set_smem_once(smem_set, kern, smem_bytes);
+  if (e != cudaSuccess) {
+    t_detail = "grouped shared-memory attribute (" + std::to_string(smem_bytes) + " bytes)";
+    return e;
+  }
+  {
+    ProfRange pr(name, st);
+    e = launch_pdl(kern, dim3((unsigned)(2 * P)), dim3(kGemmThreads), (size_t)smem_bytes, st, maps, geom);
+  }
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) t_detail = "grouped launch, " + std::to_string(tiles) + " tiles on " + std::to_string(P) + " pairs";
+  return e;
+}
+
+template <bool A_MN, bool B_MN>
+static cudaError_t grouped_bn(int bn, const GemmArgs* gs, const ClusterOut* os, int nprob, int pairs,
+                              const char* name, cudaStream_t st) {
+  if constexpr (!B_MN) {
+    if (bn == 64) return launch_grouped<PairCfg<64, A_MN, B_MN>>(gs, os, nprob, pairs, name, st);
+  }
+  if (bn == 128) return launch_grouped<PairCfg<128, A_MN, B_MN>>(gs, os, nprob, pairs, name, st);
+  if (bn == 256) return launch_grouped<PairCfg<256, A_MN, B_MN>>(gs, os, nprob, pairs, name, st);
+  if (bn == 384) return launch_grouped<PairCfg<384, A_MN, B_MN>>(gs, os, nprob, pairs, name, st);
+  if (bn == 512) return launch_grouped<PairCfg<512, A_MN, B_MN>>(gs, os, nprob, pairs, name, st);
+  t_detail = "no grouped tile of width " + std::to_string(bn);
+  return cudaErrorInvalidValue;
+}
+
 // ============================================================== operations
 
 // Gs = scale * A A^T as bf16 hi and lo halves [r x 2 rp] for a K-extension of a
@@ -1093,31 +1176,52 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     cudaError_t e = narrow_cluster<false, true>(p.du_bn, p.du_cs, a, d.s, du, r, false, st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: du");
   }
-  // dB = dz^T su  (both token-major: K = T)
-  {
-    GemmArgs a;
-    a.a0 = Mat{dz, Ti, d_out, d_out};
-    a.b0 = Mat{su, Ti, r, r};
-    a.K0 = Ti;
-    a.M = d_out;
-    a.N = r;
-    a.name = "dB_gemm";
-    cudaError_t e = narrow_cluster<true, true>(p.dB_bn, p.dB_cs, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dB), r,
-                                               false, st);
-    if (e != cudaSuccess) return gemm_status(e, "dora_backward: dB");
-  }
-  // dA^T = x^T du, stored transposed into dA [r x d_in]
-  {
-    GemmArgs a;
-    a.a0 = Mat{x, Ti, d_in, d_in};
-    a.b0 = Mat{du, Ti, r, r};
-    a.K0 = Ti;
-    a.M = d_in;
-    a.N = r;
-    a.name = "dA_gemm";
-    cudaError_t e = narrow_cluster<true, true>(p.dA_bn, p.dA_cs, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dA), d_in,
-                                               true, st);
-    if (e != cudaSuccess) return gemm_status(e, "dora_backward: dA");
+  // dB = dz^T su and dA^T = x^T du (stored transposed into dA [r x d_in]): both operands
+  // token-major, K = T. One grouped launch of whole tiles, or two cluster split-K launches
+  // when their tiles are too few for the SM pairs.
+  if (p.dBA_grouped) {
+    GemmArgs a[2];
+    a[0].a0 = Mat{dz, Ti, d_out, d_out};
+    a[0].b0 = Mat{su, Ti, r, r};
+    a[0].K0 = Ti;
+    a[0].M = d_out;
+    a[0].N = r;
+    a[1].a0 = Mat{x, Ti, d_in, d_in};
+    a[1].b0 = Mat{du, Ti, r, r};
+    a[1].K0 = Ti;
+    a[1].M = d_in;
+    a[1].N = r;
+    const ClusterOut o[2] = {{reinterpret_cast<__nv_bfloat16*>(dB), nullptr, nullptr, r, 1.0f, 0, 0},
+                             {reinterpret_cast<__nv_bfloat16*>(dA), nullptr, nullptr, d_in, 1.0f, 1, 0}};
+    cudaError_t e = grouped_bn<true, true>(p.dB_bn, a, o, 2, p.sms / 2, "dBA_gemm", st);
+    if (e != cudaSuccess) return gemm_status(e, "dora_backward: dB and dA");
+  } else {
+    // dB = dz^T su  (both token-major: K = T)
+    {
+      GemmArgs a;
+      a.a0 = Mat{dz, Ti, d_out, d_out};
+      a.b0 = Mat{su, Ti, r, r};
+      a.K0 = Ti;
+      a.M = d_out;
+      a.N = r;
+      a.name = "dB_gemm";
+      cudaError_t e = narrow_cluster<true, true>(p.dB_bn, p.dB_cs, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dB), r,
+                                                 false, st);
+      if (e != cudaSuccess) return gemm_status(e, "dora_backward: dB");
+    }
+    // dA^T = x^T du, stored transposed into dA [r x d_in]
+    {
+      GemmArgs a;
+      a.a0 = Mat{x, Ti, d_in, d_in};
+      a.b0 = Mat{du, Ti, r, r};
+      a.K0 = Ti;
+      a.M = d_in;
+      a.N = r;
+      a.name = "dA_gemm";
+      cudaError_t e = narrow_cluster<true, true>(p.dA_bn, p.dA_cs, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dA), d_in,
+                                                 true, st);
+      if (e != cudaSuccess) return gemm_status(e, "dora_backward: dA");
+    }
   }
   // dx = [dz | du] [W0 ; A]  (W0 and A read MN-major: K rows, N = d_in contiguous)
   if (dx) {

@@ -37,6 +37,8 @@ SMALL = {
     "r8_one_token": ("c2", dict(d_out=8, d_in=8, r=8, T=1)),
     "r16_wide": ("c2", dict(d_out=640, d_in=384, r=16, T=200)),
     "r64_near_unity": ("c4a", dict(d_out=384, d_in=1024, T=130)),
+    # few dB/dA tiles over a long K = T: two cluster split-K launches instead of the grouped one
+    "long_T_few_tiles": ("c4a", dict(d_out=256, d_in=512, T=16384)),
 }
 
 
