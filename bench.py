@@ -486,8 +486,13 @@ def run_ours(args, wl, cfg, dist=None, extras=True):
     if dist is not None:
         dist.barrier()
 
-    # ---- timed region: K steps, events around each step, L2 flushed before each
+    # ---- timed region: K steps, events around each step, L2 flushed before each.
+    # After each timed step (outside its events) one more step runs under the kernel
+    # profiler, also after an L2 flush, so that the per-kernel durations are taken in
+    # the same conditions (clock, power state) as the timed steps.
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    nprof = min(args.steps, 50)
+    per = {}
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
@@ -502,6 +507,12 @@ def run_ours(args, wl, cfg, dist=None, extras=True):
             if dist is not None:
                 allreduce_gradients(dm, dA, dB)
             e[4].record()
+            if i < nprof:
+                flush.zero_()
+                prof.replay()
+                torch.cuda.synchronize()
+                for name, ms in dw.dora_profile_read():
+                    per.setdefault(name, []).append(ms)
         torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
@@ -519,15 +530,6 @@ def run_ours(args, wl, cfg, dist=None, extras=True):
     ms_per_step = total_ms / args.steps
     value = world * T * args.steps / (total_ms / 1e3)
 
-    # ---- per-kernel durations from the profiled capture
-    nprof = min(args.steps, 50)
-    per = {}
-    for _ in range(nprof):
-        flush.zero_()
-        prof.replay()
-        torch.cuda.synchronize()
-        for name, ms in dw.dora_profile_read():
-            per.setdefault(name, []).append(ms)
     del prof
     peaks, peak_src = load_peaks()
     P_burst, P_sus, BW = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"], peaks["hbm_gbs"]

@@ -237,8 +237,19 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
       // off_gs directly. The norm GEMM runs on CTA pairs, 256 rows x the whole
       // rank per tile.
       p.norm_bn = bn_pair_k(r);
-      p.norm = choose_split(cdiv(d_out, 256), cdiv(d_in, 64) + 2 * cdiv(r, 64), p.sms / 2,
-                            kbB * (128 + p.norm_bn / 2.0), 0.0, (double)d_out);
+      const int64_t norm_tiles = cdiv(d_out, 256), norm_kb = cdiv(d_in, 64) + 2 * cdiv(r, 64);
+      p.norm = choose_split(norm_tiles, norm_kb, p.sms / 2, kbB * (128 + p.norm_bn / 2.0), 0.0, (double)d_out);
+      if (cdiv(r, 128) == 1 && p.sms / 2 > 8) {
+        // A single Gram tile runs beside the norm GEMM on the SMs it leaves (2 to 8 CTAs
+        // splitting K), and the norm GEMM's last split waits for it before its final
+        // k-blocks. When those SMs are too few for the Gram's K loop to finish within a
+        // split's, leave it eight.
+        const int64_t spare = p.sms - 2 * std::min<int64_t>(norm_tiles * p.norm.splits, p.sms / 2);
+        const int64_t gram_cs = spare >= 8 ? 8 : spare >= 4 ? 4 : 2;
+        if (cdiv(cdiv(d_in, 64), gram_cs) > p.norm.kb_per_split)
+          p.norm = choose_split(norm_tiles, norm_kb, p.sms / 2 - 4, kbB * (128 + p.norm_bn / 2.0), 0.0,
+                                (double)d_out);
+      }
       p.off_norm_part = take((size_t)p.norm.splits * d_out * 4);
       p.off_gs = take((size_t)r * 2 * cdiv(r, 64) * 64 * 2);
       // split counters, one per 128-row half of a pair tile, zeroed by the Gram kernel
