@@ -455,10 +455,13 @@ def run_ours(args, wl, cfg, dist=None, extras=True):
         c()
     torch.cuda.synchronize()
 
-    # One CUDA graph per call, replayed back to back between events in the timed region:
-    # the step time and the per-call times come from the same steps (each call's time
-    # includes one graph launch, ~5 us). Per-kernel times come from a capture under the
-    # library's kernel profiler (each kernel launched and timed on its own).
+    # The timed step is two CUDA graphs: the norm call (timed on its own, the metric's
+    # norm TFLOP/s) and the forward and backward calls together, as a training loop would
+    # capture them. After the timed region (and half a second idle, so that the GPU leaves
+    # the power-capped state of the timed steps) the forward and backward run again as one
+    # graph per call with events between them, for their separate times (each includes one
+    # graph launch, ~5 us), and the whole step runs under the library's kernel profiler
+    # (each kernel launched and timed on its own), each after its own L2 flush.
     def capture(fns, profiled=False):
         gph = torch.cuda.CUDAGraph()
         if profiled:
@@ -471,12 +474,17 @@ def run_ours(args, wl, cfg, dist=None, extras=True):
         torch.cuda.synchronize()
         return gph
 
-    percall = [capture([c]) for c in calls]
+    norm_graph = capture([call_norm])
+    fb_graph = capture([call_fwd, call_bwd])
+    percall = [capture([c]) for c in (call_fwd, call_bwd)]
     prof = capture(calls, profiled=True)
     launches_per_step = dw.dora_profile_count()
 
     # ---- warm-up
     for _ in range(args.warmup):
+        flush.zero_()
+        norm_graph.replay()
+        fb_graph.replay()
         flush.zero_()
         for gph in percall:
             gph.replay()
@@ -486,13 +494,8 @@ def run_ours(args, wl, cfg, dist=None, extras=True):
     if dist is not None:
         dist.barrier()
 
-    # ---- timed region: K steps, events around each step, L2 flushed before each.
-    # After each timed step (outside its events) one more step runs under the kernel
-    # profiler, also after an L2 flush, so that the per-kernel durations are taken in
-    # the same conditions (clock, power state) as the timed steps.
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    nprof = min(args.steps, 50)
-    per = {}
+    # ---- timed region: K steps, events around each step, L2 flushed before each
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
@@ -501,28 +504,43 @@ def run_ours(args, wl, cfg, dist=None, extras=True):
             flush.zero_()
             e = ev[i]
             e[0].record()
-            for k, gph in enumerate(percall):
-                gph.replay()
-                e[k + 1].record()
+            norm_graph.replay()
+            e[1].record()
+            fb_graph.replay()
+            e[2].record()
             if dist is not None:
                 allreduce_gradients(dm, dA, dB)
-            e[4].record()
-            if i < nprof:
-                flush.zero_()
-                prof.replay()
-                torch.cuda.synchronize()
-                for name, ms in dw.dora_profile_read():
-                    per.setdefault(name, []).append(ms)
+            e[3].record()
         torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    step_ms = [e[0].elapsed_time(e[4]) for e in ev]
+
+    # ---- per-call and per-kernel passes (outside the timed region)
+    time.sleep(0.5)
+    nprof = min(args.steps, 50)
+    cev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nprof)]
+    per = {}
+    for i in range(nprof):
+        flush.zero_()
+        c = cev[i]
+        c[0].record()
+        for k, gph in enumerate(percall):
+            gph.replay()
+            c[k + 1].record()
+        flush.zero_()
+        prof.replay()
+        torch.cuda.synchronize()
+        for name, ms in dw.dora_profile_read():
+            per.setdefault(name, []).append(ms)
+    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
     total_ms = sum(step_ms)
-    phase_ms = {name: statistics.mean(e[k].elapsed_time(e[k + 1]) for e in ev)
-                for k, name in enumerate(("norm", "forward", "backward"))}
+    phase_ms = {"norm": statistics.mean(e[0].elapsed_time(e[1]) for e in ev),
+                "forward": statistics.mean(c[0].elapsed_time(c[1]) for c in cev),
+                "backward": statistics.mean(c[1].elapsed_time(c[2]) for c in cev),
+                "forward_backward": statistics.mean(e[1].elapsed_time(e[2]) for e in ev)}
     if dist is not None:
-        phase_ms["allreduce"] = statistics.mean(e[3].elapsed_time(e[4]) for e in ev)
-    del percall
+        phase_ms["allreduce"] = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+    del percall, norm_graph, fb_graph
     if dist is not None:
         t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -758,7 +776,8 @@ def _table(args):
     out = ["# Layer step per workload, one B200",
            "",
            f"`python bench.py --table {os.path.basename(args.table)} --steps {args.steps} --warmup {args.warmup}`: "
-           "per workload the layer step (dora_norm + dora_forward + dora_backward, one CUDA graph per call, "
+           "per workload the layer step (dora_norm as one CUDA graph, dora_forward + dora_backward as a second; "
+           "the forward and backward times from one graph per call, after the timed region; "
            "L2 flushed before every timed step, CUDA events on the launching stream), synthetic inputs of "
            "the workload's shapes. The layer roofline is the slower of flops / measured burst bf16 peak and "
            "bytes / measured HBM copy rate per call.",
@@ -789,7 +808,8 @@ def workload_config(wl, world):
     return {"workload": wl.name, "d_out": wl.d_out, "d_in": wl.d_in, "r": wl.r, "s": wl.s,
             "tokens_per_gpu": wl.T, "global_tokens": wl.T * world, "parallelism": f"dp{world}",
             "l2": "flushed before every timed step (256 MB write)",
-            "timing": "one CUDA graph per call, CUDA events per step and call, max over ranks"}
+            "timing": "step: two CUDA graphs (norm; forward + backward) between CUDA events, max over ranks; "
+                      "call_us forward and backward: one graph per call after the timed region"}
 
 
 def main(argv=None):

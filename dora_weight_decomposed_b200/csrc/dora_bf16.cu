@@ -1091,11 +1091,12 @@ dora_status_t bf16_forward(const dora_desc_t& d, const Plan& p, int64_t T, const
   ba.split.splits = 1;
   ba.name = "fwd_compose_gemm";
   ba.split.kb_per_split = (int)(ceil_div(d_in, kBK) + ceil_div(r, kBK));
-  if (p.fwd_cs > 1) {
+  if (p.fwd_cs > 1 || p.fwd_bn != 256) {
     // Few tiles (small token batches): clusters of pairs split K and compose in the reduction.
     const ClusterOut o{reinterpret_cast<__nv_bfloat16*>(y), reinterpret_cast<__nv_bfloat16*>(pre_save), gm1, d_out,
                        1.0f, 0, 1};
-    e = pair_cluster_cs<256, false, false>(p.fwd_cs, ba, o, st);
+    e = p.fwd_bn == 128 ? pair_cluster_cs<128, false, false>(p.fwd_cs, ba, o, st)
+                        : pair_cluster_cs<256, false, false>(p.fwd_cs, ba, o, st);
     return gemm_status(e, "dora_forward: base GEMM with compose");
   }
   EpiCompose::Params cp{reinterpret_cast<__nv_bfloat16*>(y), reinterpret_cast<__nv_bfloat16*>(pre_save), gm1,
@@ -1238,9 +1239,10 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.name = "dx_gemm";
     a.split.kb_per_split = (int)(ceil_div(d_out, kBK) + ceil_div(r, kBK));
     cudaError_t e;
-    if (p.dx_cs > 1) {
+    if (p.dx_cs > 1 || p.dx_bn != 256) {
       const ClusterOut o{reinterpret_cast<__nv_bfloat16*>(dx), nullptr, nullptr, d_in, 1.0f, 0, 0};
-      e = pair_cluster_cs<256, false, true>(p.dx_cs, a, o, st);
+      e = p.dx_bn == 128 ? pair_cluster_cs<128, false, true>(p.dx_cs, a, o, st)
+                         : pair_cluster_cs<256, false, true>(p.dx_cs, a, o, st);
     } else {
       EpiStoreBF16::Params sp{reinterpret_cast<__nv_bfloat16*>(dx), d_in, 1.0f, 0};
       e = launch_gemm_pair<PairCfg<256, false, true>, EpiStoreBF16>(a, sp, p.sms, st);
