@@ -126,9 +126,31 @@ static int64_t resident_clusters(int cs, int sms) {
   return cs > 2 ? std::max<int64_t>(1, even - 3) : even;
 }
 
+static ClusterChoice choose_narrow_cluster_bn(int64_t M, int64_t N, int64_t K, int bn, int sms);
+
+// With B read K-major the rank may also be split into two column tiles (192 of r = 384,
+// 128 of r = 256): twice the tiles to spread over the SM pairs at the same k-block
+// count, for twice the reads of the A operand (from L2) per column. Chosen when the
+// time model (microseconds, as for the base GEMMs below) says so.
 static ClusterChoice choose_narrow_cluster(int64_t M, int64_t N, int64_t K, bool b_mn, int sms) {
+  const int full = b_mn ? (N <= 128 ? 128 : N <= 256 ? 256 : N <= 384 ? 384 : 512) : (int)bn_pair_k(N);
+  ClusterChoice c = choose_narrow_cluster_bn(M, N, K, full, sms);
+  const int half = N > 256 && N <= 384 ? 192 : N > 128 && N <= 256 ? 128 : 0;
+  if (b_mn || half == 0) return c;
+  const int64_t kb = std::max<int64_t>(cdiv(K, 64), 1);
+  auto us = [&](const ClusterChoice& x) {
+    const double kb_us = std::max(2.0 * 256.0 * x.bn * 64.0 / 23.0e6, (16384.0 + 64.0 * x.bn) / 110.0e3);
+    const int64_t tiles = cdiv(M, 256) * cdiv(N, x.bn);
+    return (double)cdiv(tiles, resident_clusters(x.cs, sms)) * ((double)cdiv(kb, x.cs) * kb_us + 1.5) +
+           0.75 * (x.cs - 1) * x.bn / 128.0 + 1.0;
+  };
+  const ClusterChoice h = choose_narrow_cluster_bn(M, N, K, half, sms);
+  return us(h) < us(c) ? h : c;
+}
+
+static ClusterChoice choose_narrow_cluster_bn(int64_t M, int64_t N, int64_t K, int bn, int sms) {
   ClusterChoice c;
-  c.bn = b_mn ? (N <= 128 ? 128 : N <= 256 ? 256 : N <= 384 ? 384 : 512) : (int)bn_pair_k(N);
+  c.bn = bn;
   const int64_t tiles = cdiv(M, 256) * cdiv(N, c.bn);
   const int64_t kb = std::max<int64_t>(cdiv(K, 64), 1);
   double best = 1e300;

@@ -862,6 +862,7 @@ static cudaError_t narrow_cluster(int bn, int cs, const GemmArgs& g, float alpha
   const ClusterOut o{out, nullptr, nullptr, ldo, alpha, transpose ? 1 : 0, 0};
   if constexpr (!B_MN) {
     if (bn == 64) return pair_cluster_cs<64, A_MN, B_MN>(cs, g, o, st);
+    if (bn == 192) return pair_cluster_cs<192, A_MN, B_MN>(cs, g, o, st);
   }
   if (bn == 128) return pair_cluster_cs<128, A_MN, B_MN>(cs, g, o, st);
   if (bn == 256) return pair_cluster_cs<256, A_MN, B_MN>(cs, g, o, st);
