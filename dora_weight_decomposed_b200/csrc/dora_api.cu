@@ -128,15 +128,16 @@ static int64_t resident_clusters(int cs, int sms) {
 
 static ClusterChoice choose_narrow_cluster_bn(int64_t M, int64_t N, int64_t K, int bn, int sms);
 
-// With B read K-major the rank may also be split into two column tiles (192 of r = 384,
-// 128 of r = 256): twice the tiles to spread over the SM pairs at the same k-block
-// count, for twice the reads of the A operand (from L2) per column. Chosen when the
-// time model (microseconds, as for the base GEMMs below) says so.
+// The rank may also be split into two column tiles: 192 of r = 384 or 128 of r = 256 with
+// B read K-major; with B read MN-major (whole 64-column chunks per CTA) 256 and a
+// half-empty second tile for r = 384. Twice the tiles to spread over the SM pairs at the
+// same k-block count, for twice the reads of the A operand (from L2) per column. Chosen
+// when the time model (microseconds, as for the base GEMMs below) says so.
 static ClusterChoice choose_narrow_cluster(int64_t M, int64_t N, int64_t K, bool b_mn, int sms) {
   const int full = b_mn ? (N <= 128 ? 128 : N <= 256 ? 256 : N <= 384 ? 384 : 512) : (int)bn_pair_k(N);
   ClusterChoice c = choose_narrow_cluster_bn(M, N, K, full, sms);
-  const int half = N > 256 && N <= 384 ? 192 : N > 128 && N <= 256 ? 128 : 0;
-  if (b_mn || half == 0) return c;
+  const int half = N > 256 && N <= 384 ? (b_mn ? 256 : 192) : (!b_mn && N > 128 && N <= 256) ? 128 : 0;
+  if (half == 0) return c;
   const int64_t kb = std::max<int64_t>(cdiv(K, 64), 1);
   auto us = [&](const ClusterChoice& x) {
     const double kb_us = std::max(2.0 * 256.0 * x.bn * 64.0 / 23.0e6, (16384.0 + 64.0 * x.bn) / 110.0e3);
