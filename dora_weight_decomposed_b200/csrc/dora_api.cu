@@ -155,7 +155,11 @@ static ClusterChoice choose_narrow_cluster_bn(int64_t M, int64_t N, int64_t K, i
   const int64_t tiles = cdiv(M, 256) * cdiv(N, c.bn);
   const int64_t kb = std::max<int64_t>(cdiv(K, 64), 1);
   double best = 1e300;
-  for (int cs : {1, 2, 3, 4}) {
+  // Clusters of 8 pairs (16 CTAs, a non-portable size) for tiles up to 128 columns wide,
+  // when the device reports that it can hold them.
+  const bool eight = bn <= 128 && max_active_pair_clusters(8) > 0;
+  for (int cs : {1, 2, 3, 4, 8}) {
+    if (cs == 8 && !eight) break;
     if (cs > 1 && kb < 2 * cs) break;  // at least two k-blocks per split
     const int64_t waves = cdiv(tiles, resident_clusters(cs, sms));
     const double t = (double)waves * ((double)cdiv(kb, cs) + 4.0) + (cs > 1 ? 1.0 * (cs - 1) * c.bn / 128.0 : 0.0);
@@ -167,42 +171,32 @@ static ClusterChoice choose_narrow_cluster_bn(int64_t M, int64_t N, int64_t K, i
   return c;
 }
 
-// The base GEMMs (forward, dx): the persistent pair kernel on 256 x 256 tiles, or,
-// when those tiles are too few to fill the SM pairs, clusters of 1 to 4 pairs that
-// split K on 256- or 128-wide tiles (the narrower tile doubles the tiles to spread).
-// Estimated microseconds at ~1.9 GHz: a pair k-block takes the longer of its MMAs
-// and its operand loads (~110 GB/s per SM); each wave adds 1.5 us (prologue, pipeline
-// fill, last epilogue), each extra split 0.75 us per 128 columns of reduction, and a
+// The 256 x 256 base GEMMs (forward, dx): the persistent pair kernel (1) or, when
+// its tiles are too few to fill the SM pairs, clusters of 2 to 4 pairs that split
+// K. Estimated microseconds at ~1.9 GHz: a pair k-block takes the longer of its
+// MMAs and its operand loads (~110 GB/s per SM); each wave adds 1.5 us (prologue,
+// pipeline fill, last epilogue), each extra split 1.5 us of reduction, and a
 // cluster launch 1 us for its stores. The persistent kernel overlaps each tile's
-// epilogue with the next tile's main loop, so only its waves count.
-struct WideChoice {
-  int bn = 256;
-  int cs = 1;  // 1 with bn = 256: the persistent kernel
-};
-
-static WideChoice choose_wide(int64_t M, int64_t N, int64_t K, int sms) {
+// epilogue with the next tile's main loop, so only its waves count. (256 x 128
+// cluster tiles, twice as many, measured slower: 25.2 against 22.6 us for the c4a
+// forward.)
+static int choose_wide_cs(int64_t M, int64_t N, int64_t K, int sms) {
+  const int64_t tiles = cdiv(M, 256) * cdiv(N, 256);
   const int64_t kb = std::max<int64_t>(cdiv(K, 64), 1);
   const int pairs = std::max(1, sms / 2);
-  auto kb_us = [](int bn) {
-    return std::max(2.0 * 256.0 * bn * 64.0 / 23.0e6, (16384.0 + 64.0 * bn) / 110.0e3);
-  };
-  WideChoice best;
-  double best_t = (double)cdiv(cdiv(M, 256) * cdiv(N, 256), pairs) * ((double)kb * kb_us(256) + 1.5);
-  for (int bn : {256, 128}) {
-    const int64_t tiles = cdiv(M, 256) * cdiv(N, bn);
-    for (int c : {1, 2, 3, 4}) {
-      if (bn == 256 && c == 1) continue;  // the persistent kernel above
-      if (c > 1 && kb < 2 * c) break;
-      const double t = (double)cdiv(tiles, resident_clusters(c, sms)) * ((double)cdiv(kb, c) * kb_us(bn) + 1.5) +
-                       0.75 * (c - 1) * bn / 128.0 + 1.0;
-      if (t < best_t - 1e-9) {
-        best_t = t;
-        best.bn = bn;
-        best.cs = c;
-      }
+  const double kb_us = std::max(2.0 * 256.0 * 256.0 * 64.0 / 23.0e6, (16384.0 + 64.0 * 256.0) / 110.0e3);
+  double best = (double)cdiv(tiles, pairs) * ((double)kb * kb_us + 1.5);
+  int cs = 1;
+  for (int c : {2, 3, 4}) {
+    if (kb < 2 * c) break;
+    const double t =
+        (double)cdiv(tiles, resident_clusters(c, sms)) * ((double)cdiv(kb, c) * kb_us + 1.5) + 1.5 * (c - 1) + 1.0;
+    if (t < best - 1e-9) {
+      best = t;
+      cs = c;
     }
   }
-  return best;
+  return cs;
 }
 
 // dB and dA (both K = T, tile width bn) in one grouped persistent launch of whole
@@ -299,9 +293,7 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
       const ClusterChoice u = choose_narrow_cluster(T, r, d_in, false, p.sms);
       p.u_bn = u.bn;
       p.u_cs = u.cs;
-      const WideChoice fw = choose_wide(T, d_out, cdiv(d_in, 64) * 64 + cdiv(r, 64) * 64, p.sms);
-      p.fwd_bn = fw.bn;
-      p.fwd_cs = fw.cs;
+      p.fwd_cs = choose_wide_cs(T, d_out, cdiv(d_in, 64) * 64 + cdiv(r, 64) * 64, p.sms);
       p.off_su = take((size_t)T * r * 2);
     } else if ((op == DORA_OP_BACKWARD || op == DORA_OP_BACKWARD_FULL) && T > 0) {
       p.off_dz = take((size_t)T * d_out * 2);
@@ -325,9 +317,7 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
       p.dA_bn = dA.bn;
       p.dA_cs = dA.cs;
       p.dBA_grouped = dBA_grouped(d_out, d_in, r, T, p.dB_bn, p.sms) ? 1 : 0;
-      const WideChoice xw = choose_wide(T, d_in, cdiv(d_out, 64) * 64 + cdiv(r, 64) * 64, p.sms);
-      p.dx_bn = xw.bn;
-      p.dx_cs = xw.cs;
+      p.dx_cs = choose_wide_cs(T, d_in, cdiv(d_out, 64) * 64 + cdiv(r, 64) * 64, p.sms);
       // counters of the dm column strips, zeroed by one memset per call
       p.zero_bytes = (size_t)cdiv(d_out, 64) * 4;
       p.off_ctr = take(p.zero_bytes);

@@ -747,8 +747,9 @@ static cudaError_t launch_pair_cluster(const GemmArgs& g, const ClusterOut& o, c
   constexpr int smem_bytes = PairClusterLayout<Cfg>::SMEM_BYTES;
   static std::atomic<unsigned long long> smem_set{0};
   cudaError_t e = set_smem_once(smem_set, kern, smem_bytes);
+  if (e == cudaSuccess && CS > 4) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e != cudaSuccess) {
-    t_detail = "shared-memory attribute (" + std::to_string(smem_bytes) + " bytes)";
+    t_detail = "shared-memory or cluster-size attribute (" + std::to_string(smem_bytes) + " bytes)";
     return e;
   }
   cudaLaunchConfig_t cfg = {};
@@ -783,6 +784,9 @@ static cudaError_t pair_cluster_cs(int cs, const GemmArgs& g, const ClusterOut& 
   if (cs == 2) return launch_pair_cluster<Cfg, 2>(g, o, st);
   if (cs == 3) return launch_pair_cluster<Cfg, 3>(g, o, st);
   if (cs == 4) return launch_pair_cluster<Cfg, 4>(g, o, st);
+  if constexpr (BN <= 128) {
+    if (cs == 8) return launch_pair_cluster<Cfg, 8>(g, o, st);
+  }
   t_detail = "no cluster of " + std::to_string(cs) + " pairs";
   return cudaErrorInvalidValue;
 }
@@ -792,8 +796,8 @@ static cudaError_t pair_cluster_cs(int cs, const GemmArgs& g, const ClusterOut& 
 // below SMs / (2 cs) for the larger clusters (e.g. 15 clusters of 8 CTAs on a
 // 148-SM B200). Queried once per device and cluster size; 0 if the query fails.
 int max_active_pair_clusters(int cs) {
-  static std::atomic<int> cache[64][5];
-  if (cs < 1 || cs > 4) return 0;
+  static std::atomic<int> cache[64][9];
+  if (cs < 1 || (cs > 4 && cs != 8)) return 0;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     cudaGetLastError();
@@ -838,10 +842,22 @@ int max_active_pair_clusters(int cs) {
       if (e == cudaSuccess) e = cudaOccupancyMaxActiveClusters(&n, k, &cfg);
       break;
     }
-    default: {
+    case 4: {
       static std::atomic<unsigned long long> set{0};
       auto k = gemm_sm100_pair_cluster_kernel<Cfg, 4>;
       e = set_smem_once(set, k, smem_bytes);
+      if (e == cudaSuccess) e = cudaOccupancyMaxActiveClusters(&n, k, &cfg);
+      break;
+    }
+    default: {
+      // 16-CTA clusters (non-portable), used with tiles up to 128 columns wide only.
+      using Cfg8 = PairCfg<128, false, false>;
+      constexpr int smem8 = PairClusterLayout<Cfg8>::SMEM_BYTES;
+      cfg.dynamicSmemBytes = smem8;
+      static std::atomic<unsigned long long> set{0};
+      auto k = gemm_sm100_pair_cluster_kernel<Cfg8, 8>;
+      e = set_smem_once(set, k, smem8);
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
       if (e == cudaSuccess) e = cudaOccupancyMaxActiveClusters(&n, k, &cfg);
       break;
     }
@@ -1092,12 +1108,11 @@ dora_status_t bf16_forward(const dora_desc_t& d, const Plan& p, int64_t T, const
   ba.split.splits = 1;
   ba.name = "fwd_compose_gemm";
   ba.split.kb_per_split = (int)(ceil_div(d_in, kBK) + ceil_div(r, kBK));
-  if (p.fwd_cs > 1 || p.fwd_bn != 256) {
+  if (p.fwd_cs > 1) {
     // Few tiles (small token batches): clusters of pairs split K and compose in the reduction.
     const ClusterOut o{reinterpret_cast<__nv_bfloat16*>(y), reinterpret_cast<__nv_bfloat16*>(pre_save), gm1, d_out,
                        1.0f, 0, 1};
-    e = p.fwd_bn == 128 ? pair_cluster_cs<128, false, false>(p.fwd_cs, ba, o, st)
-                        : pair_cluster_cs<256, false, false>(p.fwd_cs, ba, o, st);
+    e = pair_cluster_cs<256, false, false>(p.fwd_cs, ba, o, st);
     return gemm_status(e, "dora_forward: base GEMM with compose");
   }
   EpiCompose::Params cp{reinterpret_cast<__nv_bfloat16*>(y), reinterpret_cast<__nv_bfloat16*>(pre_save), gm1,
@@ -1240,10 +1255,9 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.name = "dx_gemm";
     a.split.kb_per_split = (int)(ceil_div(d_out, kBK) + ceil_div(r, kBK));
     cudaError_t e;
-    if (p.dx_cs > 1 || p.dx_bn != 256) {
+    if (p.dx_cs > 1) {
       const ClusterOut o{reinterpret_cast<__nv_bfloat16*>(dx), nullptr, nullptr, d_in, 1.0f, 0, 0};
-      e = p.dx_bn == 128 ? pair_cluster_cs<128, false, true>(p.dx_cs, a, o, st)
-                         : pair_cluster_cs<256, false, true>(p.dx_cs, a, o, st);
+      e = pair_cluster_cs<256, false, true>(p.dx_cs, a, o, st);
     } else {
       EpiStoreBF16::Params sp{reinterpret_cast<__nv_bfloat16*>(dx), d_in, 1.0f, 0};
       e = launch_gemm_pair<PairCfg<256, false, true>, EpiStoreBF16>(a, sp, p.sms, st);

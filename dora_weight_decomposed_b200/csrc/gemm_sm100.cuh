@@ -852,7 +852,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 //
 // For GEMMs whose output tiles are too few to fill the GPU (the narrow rank-r
 // GEMMs with N = r and a long K, and the base GEMMs of small token batches): a
-// cluster of 2 * CS CTAs, i.e. CS CTA pairs, computes one 256 x BN output
+// cluster of 2 * CS CTAs, i.e. CS CTA pairs (1 to 4, or 8: 16 CTAs, a cluster
+// size B200 allows as non-portable), computes one 256 x BN output
 // tile, pair z (cluster ranks 2z and 2z + 1) taking the z-th K range. K may
 // come from two sources back to back, as in the other kernels. Each pair runs
 // the pair kernels' main loop (its leader is rank 2z; commits go to the pair's
@@ -895,7 +896,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_sm100_pair_cluster_kernel(const __grid_constant__ CUtensorMap tA0, const __grid_constant__ CUtensorMap tA1,
                                    const __grid_constant__ CUtensorMap tB0, const __grid_constant__ CUtensorMap tB1,
                                    const GemmGeom geom, const ClusterOut o) {
-  static_assert(CS >= 1 && CS <= 4, "pairs per cluster");
+  static_assert((CS >= 1 && CS <= 4) || CS == 8, "pairs per cluster");
   using L = PairClusterLayout<Cfg>;
   constexpr int STAGES = L::STAGES;
   constexpr int CW = L::CW;
@@ -1085,7 +1086,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (!o.transpose) {
       // item = (row, 4 columns): out[m][n .. n + 3]. kU items per thread per batch: all
       // their loads are issued before any is summed (kU * CS reads in flight).
-      constexpr int kU = 4;
+      constexpr int kU = CS > 4 ? 2 : 4;
       const int per_row = cw / 4;
       const int n_items = rows * per_row;
 #pragma unroll 1
@@ -1131,34 +1132,46 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
     } else {
-      // item = (4 columns, 8 rows): out[n .. n + 3][m .. m + 7]; its 8 CS loads are all
-      // issued before any is summed.
+      // item = (4 columns, 8 rows): out[n .. n + 3][m .. m + 7]; the 8 loads of up to four
+      // splits are issued before any is summed, the splits added in order.
+      constexpr int ZC = CS < 4 ? CS : 4;
       const int quads = cw / 4;
       const int n_items = (rows / 8) * quads;
 #pragma unroll 1
       for (int it = threadIdx.x; it < n_items; it += kGemmThreads) {
         const int lc = (it % quads) * 4;
         const int lr = row_lo + (it / quads) * 8;
-        float4 x[CS][8];
+        float4 v[8];
 #pragma unroll
-        for (int zz = 0; zz < CS; ++zz)
+        for (int zz0 = 0; zz0 < CS; zz0 += ZC) {
+          float4 x[ZC][8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) x[zz][i] = *reinterpret_cast<const float4*>(srcs[zz] + (lr + i) * RS + lc);
+          for (int zz = 0; zz < ZC; ++zz)
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              x[zz][i] = *reinterpret_cast<const float4*>(srcs[zz0 + zz] + (lr + i) * RS + lc);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+#pragma unroll
+            for (int zz = 0; zz < ZC; ++zz) {
+              if (zz0 + zz == 0) {
+                v[i] = x[0][i];
+              } else {
+                v[i].x += x[zz][i].x;
+                v[i].y += x[zz][i].y;
+                v[i].z += x[zz][i].z;
+                v[i].w += x[zz][i].w;
+              }
+            }
+          }
+        }
         float a[4][8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          float4 v = x[0][i];
-#pragma unroll
-          for (int zz = 1; zz < CS; ++zz) {
-            v.x += x[zz][i].x;
-            v.y += x[zz][i].y;
-            v.z += x[zz][i].z;
-            v.w += x[zz][i].w;
-          }
-          a[0][i] = o.alpha * v.x;
-          a[1][i] = o.alpha * v.y;
-          a[2][i] = o.alpha * v.z;
-          a[3][i] = o.alpha * v.w;
+          a[0][i] = o.alpha * v[i].x;
+          a[1][i] = o.alpha * v[i].y;
+          a[2][i] = o.alpha * v[i].z;
+          a[3][i] = o.alpha * v[i].w;
         }
         const int m = m0 + lr;
         const int n = tn * Cfg::BN + c0 + lc;
