@@ -39,6 +39,9 @@ SMALL = {
     "r64_near_unity": ("c4a", dict(d_out=384, d_in=1024, T=130)),
     # few dB/dA tiles over a long K = T: two cluster split-K launches instead of the grouped one
     "long_T_few_tiles": ("c4a", dict(d_out=256, d_in=512, T=16384)),
+    # 74 + 2 grouped dB/dA tiles of 256 x 128: more tiles than SM pairs, so pairs run two tiles
+    # through the grouped kernel's two TMEM accumulators
+    "grouped_two_waves": ("c4a", dict(d_out=18944, d_in=512, T=64)),
 }
 
 
