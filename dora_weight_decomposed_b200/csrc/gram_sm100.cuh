@@ -179,15 +179,22 @@ __global__ void __launch_bounds__(192, 1) gram_cluster_kernel(const __grid_const
                     kGramTrOffset + 2 * kGramTile * kTrLd * 2 <= kGramStages * kGramStageBytes,
                 "transposed staging fits the ring after the fp32 buffer");
   // Four items per thread per batch: all their remote loads are issued before any is summed.
-  constexpr int kItems = kRows * (kGramTile / 4);
+  // A single tile (r <= 128, diagonal, nothing to transpose) spreads only its r valid rows and
+  // rp columns over the cluster, so small ranks do not reduce the zero padding of the tile.
+  const bool single = p.nt == 1;
+  const int rows_per = single ? (p.r + CS - 1) / CS : kRows;
+  const int row_lo = (int)crank * rows_per;
+  const int rows_here = single ? max(0, min(p.r, row_lo + rows_per) - row_lo) : kRows;
+  const int cols4 = single ? p.rp / 4 : kGramTile / 4;  // 4-column items per row
+  const int n_items = rows_here * cols4;
   constexpr int kU = 4;
-  for (int idx0 = threadIdx.x; idx0 < kItems; idx0 += 192 * kU) {
+  for (int idx0 = threadIdx.x; idx0 < n_items; idx0 += 192 * kU) {
     float4 vv[kU][CS];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int idx = idx0 + u * 192;
-      if (idx < kItems) {
-        const int off = ((int)crank * kRows + idx / (kGramTile / 4)) * kGramRedLd + (idx % (kGramTile / 4)) * 4;
+      if (idx < n_items) {
+        const int off = (row_lo + idx / cols4) * kGramRedLd + (idx % cols4) * 4;
 #pragma unroll
         for (int z = 0; z < CS; ++z) vv[u][z] = *reinterpret_cast<const float4*>(srcs[z] + off);
       }
@@ -195,9 +202,9 @@ __global__ void __launch_bounds__(192, 1) gram_cluster_kernel(const __grid_const
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int idx = idx0 + u * 192;
-      if (idx >= kItems) break;
-      const int lr = (int)crank * kRows + idx / (kGramTile / 4);
-      const int lc = (idx % (kGramTile / 4)) * 4;
+      if (idx >= n_items) break;
+      const int lr = row_lo + idx / cols4;
+      const int lc = (idx % cols4) * 4;
       float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int z = 0; z < CS; ++z) {
@@ -219,7 +226,7 @@ __global__ void __launch_bounds__(192, 1) gram_cluster_kernel(const __grid_const
       }
       if (!diag) {
         // The transposed values, staged so that tile (tj, ti) is written in whole rows below.
-        const int lrl = lr - (int)crank * kRows;
+        const int lrl = lr - row_lo;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           tr_hi[(lc + j) * kTrLd + lrl] = hi[j];
