@@ -221,6 +221,46 @@ static bool dBA_grouped(int64_t d_out, int64_t d_in, int64_t r, int64_t T, int b
   return grouped <= clustered(tB) + clustered(tA);
 }
 
+// dx and the grouped dB/dA launch read only dz, du and the inputs, and write disjoint
+// outputs: both may run at once. When dx's persistent tiles fit on fewer pairs than the
+// device has without another wave (or its clusters leave pairs idle), dB/dA takes the
+// idle pairs on a second stream, provided its estimate (as in dBA_grouped) stays under
+// dx's (as in choose_wide_cs); the step then loses the dB/dA launch from its critical path.
+static void plan_backward_fork(Plan& p, int64_t d_out, int64_t d_in, int64_t r, int64_t T) {
+  const int pairs = std::max(1, p.sms / 2);
+  p.bwd_fork = 0;
+  p.dx_pairs = pairs;
+  p.dBA_pairs = pairs;
+  if (!p.dBA_grouped) return;
+  // pairs the device can place at once (a GPC with an odd SM count strands one SM)
+  const int64_t placeable = std::min<int64_t>(pairs, resident_clusters(1, p.sms));
+  const int64_t tiles = cdiv(T, 256) * cdiv(d_in, 256);
+  const int64_t kb = std::max<int64_t>(cdiv(d_out, 64) + cdiv(r, 64), 1);
+  const double kb_us = std::max(2.0 * 256.0 * 256.0 * 64.0 / 23.0e6, (16384.0 + 64.0 * 256.0) / 110.0e3);
+  int64_t used;
+  double dx_us;
+  if (p.dx_cs == 1) {
+    const int64_t waves = cdiv(tiles, pairs);
+    used = cdiv(tiles, waves);
+    dx_us = (double)waves * ((double)kb * kb_us + 1.5);
+  } else {
+    const int64_t rc = resident_clusters(p.dx_cs, p.sms);
+    used = std::min(tiles, rc) * p.dx_cs;
+    dx_us = (double)cdiv(tiles, rc) * ((double)cdiv(kb, p.dx_cs) * kb_us + 1.5) + 1.5 * (p.dx_cs - 1) + 1.0;
+  }
+  const int64_t idle = placeable - used;
+  if (idle < 1) return;
+  const int bn = p.dB_bn;
+  const int64_t kbT = std::max<int64_t>(cdiv(T, 64), 1);
+  const double kbT_us = std::max(2.0 * 256.0 * bn * 64.0 / 23.0e6, (16384.0 + 64.0 * bn) / 110.0e3);
+  const int64_t tBA = (cdiv(d_out, 256) + cdiv(d_in, 256)) * cdiv(r, bn);
+  const double dBA_us = (double)cdiv(tBA, idle) * (double)kbT * kbT_us + 4.0;
+  if (dBA_us > dx_us) return;
+  p.bwd_fork = 1;
+  p.dx_pairs = (int)used;
+  p.dBA_pairs = (int)std::min(idle, tBA);
+}
+
 static NarrowChoice choose_narrow(int64_t M, int64_t N, int64_t K, bool b_mn, int sms) {
   static const int kCandK[] = {64, 128, 256, 384, 512};
   static const int kCandMN[] = {128, 256, 384, 512};
@@ -318,6 +358,7 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
       p.dA_cs = dA.cs;
       p.dBA_grouped = dBA_grouped(d_out, d_in, r, T, p.dB_bn, p.sms) ? 1 : 0;
       p.dx_cs = choose_wide_cs(T, d_in, cdiv(d_out, 64) * 64 + cdiv(r, 64) * 64, p.sms);
+      plan_backward_fork(p, d_out, d_in, r, T);
       // counters of the dm column strips, zeroed by one memset per call
       p.zero_bytes = (size_t)cdiv(d_out, 64) * 4;
       p.off_ctr = take(p.zero_bytes);

@@ -1149,6 +1149,130 @@ dora_status_t bf16_merge(const dora_desc_t& d, const Plan& p, const void* W0, co
   return gemm_status(e, "dora_merge");
 }
 
+// dB = dz^T su and dA^T = x^T du (stored transposed into dA [r x d_in]): both operands
+// token-major, K = T. One grouped launch of whole tiles on `pairs` SM pairs, or two
+// cluster split-K launches when their tiles are too few for the SM pairs.
+static dora_status_t backward_dBA(const Plan& p, int Ti, int d_out, int d_in, int r, const __nv_bfloat16* dz,
+                                  const void* su, const void* x, const __nv_bfloat16* du, void* dA, void* dB,
+                                  int pairs, cudaStream_t st) {
+  if (p.dBA_grouped) {
+    GemmArgs a[2];
+    a[0].a0 = Mat{dz, Ti, d_out, d_out};
+    a[0].b0 = Mat{su, Ti, r, r};
+    a[0].K0 = Ti;
+    a[0].M = d_out;
+    a[0].N = r;
+    a[1].a0 = Mat{x, Ti, d_in, d_in};
+    a[1].b0 = Mat{du, Ti, r, r};
+    a[1].K0 = Ti;
+    a[1].M = d_in;
+    a[1].N = r;
+    const ClusterOut o[2] = {{reinterpret_cast<__nv_bfloat16*>(dB), nullptr, nullptr, r, 1.0f, 0, 0},
+                             {reinterpret_cast<__nv_bfloat16*>(dA), nullptr, nullptr, d_in, 1.0f, 1, 0}};
+    cudaError_t e = grouped_bn<true, true>(p.dB_bn, a, o, 2, pairs, "dBA_gemm", st);
+    if (e != cudaSuccess) return gemm_status(e, "dora_backward: dB and dA");
+  } else {
+    // dB = dz^T su  (both token-major: K = T)
+    {
+      GemmArgs a;
+      a.a0 = Mat{dz, Ti, d_out, d_out};
+      a.b0 = Mat{su, Ti, r, r};
+      a.K0 = Ti;
+      a.M = d_out;
+      a.N = r;
+      a.name = "dB_gemm";
+      cudaError_t e = narrow_cluster<true, true>(p.dB_bn, p.dB_cs, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dB), r,
+                                                 false, st);
+      if (e != cudaSuccess) return gemm_status(e, "dora_backward: dB");
+    }
+    // dA^T = x^T du, stored transposed into dA [r x d_in]
+    {
+      GemmArgs a;
+      a.a0 = Mat{x, Ti, d_in, d_in};
+      a.b0 = Mat{du, Ti, r, r};
+      a.K0 = Ti;
+      a.M = d_in;
+      a.N = r;
+      a.name = "dA_gemm";
+      cudaError_t e = narrow_cluster<true, true>(p.dA_bn, p.dA_cs, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dA), d_in,
+                                                 true, st);
+      if (e != cudaSuccess) return gemm_status(e, "dora_backward: dA");
+    }
+  }
+  return DORA_OK;
+}
+
+// dx = [dz | du] [W0 ; A]  (W0 and A read MN-major: K rows, N = d_in contiguous); the
+// persistent kernel on at most sms / 2 pairs.
+static dora_status_t backward_dx(const Plan& p, int Ti, int d_out, int d_in, int r, const __nv_bfloat16* dz,
+                                 const __nv_bfloat16* du, const void* W0, const void* A, void* dx, int sms,
+                                 cudaStream_t st) {
+  {
+    GemmArgs a;
+    a.a0 = Mat{dz, Ti, d_out, d_out};
+    a.a1 = Mat{du, Ti, r, r};
+    a.b0 = Mat{W0, d_out, d_in, d_in};
+    a.b1 = Mat{A, r, d_in, d_in};
+    a.K0 = d_out;
+    a.K1 = r;
+    a.M = Ti;
+    a.N = d_in;
+    a.split.splits = 1;
+    a.name = "dx_gemm";
+    a.split.kb_per_split = (int)(ceil_div(d_out, kBK) + ceil_div(r, kBK));
+    cudaError_t e;
+    if (p.dx_cs > 1) {
+      const ClusterOut o{reinterpret_cast<__nv_bfloat16*>(dx), nullptr, nullptr, d_in, 1.0f, 0, 0};
+      e = pair_cluster_cs<256, false, true>(p.dx_cs, a, o, st);
+    } else {
+      EpiStoreBF16::Params sp{reinterpret_cast<__nv_bfloat16*>(dx), d_in, 1.0f, 0};
+      e = launch_gemm_pair<PairCfg<256, false, true>, EpiStoreBF16>(a, sp, sms, st);
+    }
+    if (e != cudaSuccess) return gemm_status(e, "dora_backward: dx");
+  }
+  return DORA_OK;
+}
+
+// The backward's second stream, with its fork and join events: one set per thread and
+// device, created on first use outside a stream capture (creating them inside one is not
+// allowed in every capture mode) and kept for the life of the thread.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+static SideStream* side_stream(cudaStream_t st) {
+  constexpr int kMaxDevices = 64;
+  thread_local SideStream per_device[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  SideStream& ss = per_device[dev];
+  if (ss.s != nullptr) return &ss;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  cudaStream_t s = nullptr;
+  cudaEvent_t f = nullptr, j = nullptr;
+  if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&f, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&j, cudaEventDisableTiming) != cudaSuccess) {
+    (void)cudaGetLastError();
+    if (j) cudaEventDestroy(j);
+    if (f) cudaEventDestroy(f);
+    if (s) cudaStreamDestroy(s);
+    return nullptr;
+  }
+  ss.s = s;
+  ss.fork = f;
+  ss.join = j;
+  return &ss;
+}
+
 dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, const void* dy, const void* x,
                             const void* W0, const void* A, const void* B, const float* C, const float* g,
                             const void* su, const void* pre, float* dm, void* dA, void* dB, void* dx,
@@ -1193,78 +1317,29 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     cudaError_t e = narrow_cluster<false, true>(p.du_bn, p.du_cs, a, d.s, du, r, false, st);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: du");
   }
-  // dB = dz^T su and dA^T = x^T du (stored transposed into dA [r x d_in]): both operands
-  // token-major, K = T. One grouped launch of whole tiles, or two cluster split-K launches
-  // when their tiles are too few for the SM pairs.
-  if (p.dBA_grouped) {
-    GemmArgs a[2];
-    a[0].a0 = Mat{dz, Ti, d_out, d_out};
-    a[0].b0 = Mat{su, Ti, r, r};
-    a[0].K0 = Ti;
-    a[0].M = d_out;
-    a[0].N = r;
-    a[1].a0 = Mat{x, Ti, d_in, d_in};
-    a[1].b0 = Mat{du, Ti, r, r};
-    a[1].K0 = Ti;
-    a[1].M = d_in;
-    a[1].N = r;
-    const ClusterOut o[2] = {{reinterpret_cast<__nv_bfloat16*>(dB), nullptr, nullptr, r, 1.0f, 0, 0},
-                             {reinterpret_cast<__nv_bfloat16*>(dA), nullptr, nullptr, d_in, 1.0f, 1, 0}};
-    cudaError_t e = grouped_bn<true, true>(p.dB_bn, a, o, 2, p.sms / 2, "dBA_gemm", st);
-    if (e != cudaSuccess) return gemm_status(e, "dora_backward: dB and dA");
-  } else {
-    // dB = dz^T su  (both token-major: K = T)
-    {
-      GemmArgs a;
-      a.a0 = Mat{dz, Ti, d_out, d_out};
-      a.b0 = Mat{su, Ti, r, r};
-      a.K0 = Ti;
-      a.M = d_out;
-      a.N = r;
-      a.name = "dB_gemm";
-      cudaError_t e = narrow_cluster<true, true>(p.dB_bn, p.dB_cs, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dB), r,
-                                                 false, st);
-      if (e != cudaSuccess) return gemm_status(e, "dora_backward: dB");
-    }
-    // dA^T = x^T du, stored transposed into dA [r x d_in]
-    {
-      GemmArgs a;
-      a.a0 = Mat{x, Ti, d_in, d_in};
-      a.b0 = Mat{du, Ti, r, r};
-      a.K0 = Ti;
-      a.M = d_in;
-      a.N = r;
-      a.name = "dA_gemm";
-      cudaError_t e = narrow_cluster<true, true>(p.dA_bn, p.dA_cs, a, 1.0f, reinterpret_cast<__nv_bfloat16*>(dA), d_in,
-                                                 true, st);
-      if (e != cudaSuccess) return gemm_status(e, "dora_backward: dA");
-    }
+  // dx and dB/dA both follow du and nothing else. Under the plan's fork dx goes to the
+  // second stream, on the pairs its tiles need, and the grouped dB/dA launch takes the
+  // idle pairs beside it; the caller's stream waits for both before this call returns.
+  // (Serial when the kernel profiler times each launch on its own.)
+  SideStream* side = (p.bwd_fork && dx && !profiling_on()) ? side_stream(st) : nullptr;
+  if (!side) {
+    const dora_status_t status = backward_dBA(p, Ti, d_out, d_in, r, dz, su, x, du, dA, dB, p.sms / 2, st);
+    if (status != DORA_OK || !dx) return status;
+    return backward_dx(p, Ti, d_out, d_in, r, dz, du, W0, A, dx, p.sms, st);
   }
-  // dx = [dz | du] [W0 ; A]  (W0 and A read MN-major: K rows, N = d_in contiguous)
-  if (dx) {
-    GemmArgs a;
-    a.a0 = Mat{dz, Ti, d_out, d_out};
-    a.a1 = Mat{du, Ti, r, r};
-    a.b0 = Mat{W0, d_out, d_in, d_in};
-    a.b1 = Mat{A, r, d_in, d_in};
-    a.K0 = d_out;
-    a.K1 = r;
-    a.M = Ti;
-    a.N = d_in;
-    a.split.splits = 1;
-    a.name = "dx_gemm";
-    a.split.kb_per_split = (int)(ceil_div(d_out, kBK) + ceil_div(r, kBK));
-    cudaError_t e;
-    if (p.dx_cs > 1) {
-      const ClusterOut o{reinterpret_cast<__nv_bfloat16*>(dx), nullptr, nullptr, d_in, 1.0f, 0, 0};
-      e = pair_cluster_cs<256, false, true>(p.dx_cs, a, o, st);
-    } else {
-      EpiStoreBF16::Params sp{reinterpret_cast<__nv_bfloat16*>(dx), d_in, 1.0f, 0};
-      e = launch_gemm_pair<PairCfg<256, false, true>, EpiStoreBF16>(a, sp, p.sms, st);
-    }
-    if (e != cudaSuccess) return gemm_status(e, "dora_backward: dx");
+  {
+    cudaError_t e = cudaEventRecord(side->fork, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s, side->fork, 0);
+    if (e != cudaSuccess) return cuda_status(e, "dora_backward: forking dx onto the second stream");
   }
-  return DORA_OK;
+  const dora_status_t dBA_status = backward_dBA(p, Ti, d_out, d_in, r, dz, su, x, du, dA, dB, p.dBA_pairs, st);
+  const dora_status_t dx_status = backward_dx(p, Ti, d_out, d_in, r, dz, du, W0, A, dx, 2 * p.dx_pairs, side->s);
+  {
+    cudaError_t e = cudaEventRecord(side->join, side->s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, side->join, 0);
+    if (e != cudaSuccess) return cuda_status(e, "dora_backward: joining the second stream");
+  }
+  return dBA_status != DORA_OK ? dBA_status : dx_status;
 }
 
 // Full (non-detached) gradient: the detached backward, then per row the

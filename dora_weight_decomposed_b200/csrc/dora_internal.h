@@ -33,6 +33,9 @@ struct Plan {
   int dm_rowblocks = 0, dm_rows = 256;
   // (dB_grouped: dB and dA in one grouped launch of whole tiles, both dB_bn wide)
   int du_bn = 0, du_cs = 1, dB_bn = 0, dB_cs = 1, dA_bn = 0, dA_cs = 1, dx_cs = 1, dBA_grouped = 0;
+  // dx and the grouped dB/dA launch both follow du alone; when dx's tiles leave SM pairs
+  // free (bwd_fork), dx runs on a second stream on dx_pairs pairs, dB/dA beside it on dBA_pairs
+  int bwd_fork = 0, dx_pairs = 0, dBA_pairs = 0;
   size_t off_dz = 0, off_dm_part = 0, off_du = 0;
   // full (non-detached) gradient: kappa, kappa-scaled B, Gram, Q = W' A^T, H = s B^T diag(kappa) B
   Split q, h;
