@@ -13,9 +13,10 @@ Under torchrun (N > 1) every rank runs the step on its own tokens with
 replicated weights and the per-rank dm, dA, dB are summed with NCCL (weak
 scaling). Rank 0 prints one JSON line.
 
-Timing: the three calls are captured into CUDA graphs (one per call) and each
-timed step replays them between CUDA events, after a 256 MB L2 flush outside
-the events. Kernel durations come from the library's own event profiler on a
+Timing: each timed step replays one CUDA graph of the three calls between
+CUDA events, after a 256 MB L2 flush outside the events. After the timed
+region each call is timed on its own (the norm call by event nodes inside a
+graph of that call alone), each after its own L2 flush. Kernel durations come from the library's own event profiler on a
 second, profiled capture of the same calls. `e2e` runs the public Python API
 eagerly with every step's inputs copied from pinned host memory and its
 results copied back inside the timed region, the copies of neighbouring steps
@@ -455,27 +456,35 @@ def run_ours(args, wl, cfg, dist=None, extras=True):
         c()
     torch.cuda.synchronize()
 
-    # The timed step is two CUDA graphs: the norm call (timed on its own, the metric's
-    # norm TFLOP/s) and the forward and backward calls together, as a training loop would
-    # capture them. After the timed region (and half a second idle, so that the GPU leaves
-    # the power-capped state of the timed steps) the forward and backward run again as one
-    # graph per call with events between them, for their separate times (each includes one
-    # graph launch, ~5 us), and the whole step runs under the library's kernel profiler
-    # (each kernel launched and timed on its own), each after its own L2 flush.
-    def capture(fns, profiled=False):
+    # The timed step is one CUDA graph holding the three calls, as a training loop would capture
+    # its step (kernel to kernel, each one's prologue overlapping its predecessor's tail). After the
+    # timed region (and half a second idle, so that the GPU leaves the power-capped state of the
+    # timed steps) each call is timed on its own, after its own L2 flush: the norm call (the
+    # metric's norm TFLOP/s) by two event record nodes inside a graph of that call alone (events
+    # made with external=True), so that its time leaves out the graph's launch; the forward and
+    # backward as one graph per call with events between them (each time includes one graph launch,
+    # ~3 us). The whole step also runs under the library's kernel profiler (each kernel launched and
+    # timed on its own). (Event nodes inside the step's own graph would time the norm there too, but
+    # each cost the step ~3 us: 98.0 against 95.2 us at c4a.)
+    def capture(fns, profiled=False, marks=None):
         gph = torch.cuda.CUDAGraph()
         if profiled:
             dw.dora_profile_start(256)
         with torch.cuda.graph(gph):
+            if marks is not None:
+                marks[0].record()
             for c in fns:
                 c()
+            if marks is not None:
+                marks[1].record()
         if profiled:
             dw.dora_profile_stop()
         torch.cuda.synchronize()
         return gph
 
-    norm_graph = capture([call_norm])
-    fb_graph = capture([call_fwd, call_bwd])
+    step_graph = capture(calls)
+    norm_marks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+    norm_marked = capture([call_norm], marks=norm_marks)
     percall = [capture([c]) for c in (call_fwd, call_bwd)]
     prof = capture(calls, profiled=True)
     launches_per_step = dw.dora_profile_count()
@@ -483,9 +492,9 @@ def run_ours(args, wl, cfg, dist=None, extras=True):
     # ---- warm-up
     for _ in range(args.warmup):
         flush.zero_()
-        norm_graph.replay()
-        fb_graph.replay()
+        step_graph.replay()
         flush.zero_()
+        norm_marked.replay()
         for gph in percall:
             gph.replay()
         if dist is not None:
@@ -495,7 +504,7 @@ def run_ours(args, wl, cfg, dist=None, extras=True):
         dist.barrier()
 
     # ---- timed region: K steps, events around each step, L2 flushed before each
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
@@ -504,13 +513,11 @@ def run_ours(args, wl, cfg, dist=None, extras=True):
             flush.zero_()
             e = ev[i]
             e[0].record()
-            norm_graph.replay()
+            step_graph.replay()
             e[1].record()
-            fb_graph.replay()
-            e[2].record()
             if dist is not None:
                 allreduce_gradients(dm, dA, dB)
-            e[3].record()
+            e[2].record()
         torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
@@ -520,7 +527,12 @@ def run_ours(args, wl, cfg, dist=None, extras=True):
     nprof = min(args.steps, 50)
     cev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nprof)]
     per = {}
+    norm_ms = []
     for i in range(nprof):
+        flush.zero_()
+        norm_marked.replay()
+        torch.cuda.synchronize()
+        norm_ms.append(norm_marks[0].elapsed_time(norm_marks[1]))
         flush.zero_()
         c = cev[i]
         c[0].record()
@@ -532,17 +544,16 @@ def run_ours(args, wl, cfg, dist=None, extras=True):
         torch.cuda.synchronize()
         for name, ms in dw.dora_profile_read():
             per.setdefault(name, []).append(ms)
-    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
     total_ms = sum(step_ms)
-    phase_ms = {"norm": statistics.mean(e[0].elapsed_time(e[1]) for e in ev),
+    phase_ms = {"norm": statistics.mean(norm_ms),
                 "forward": statistics.mean(c[0].elapsed_time(c[1]) for c in cev),
-                "backward": statistics.mean(c[1].elapsed_time(c[2]) for c in cev),
-                "forward_backward": statistics.mean(e[1].elapsed_time(e[2]) for e in ev)}
+                "backward": statistics.mean(c[1].elapsed_time(c[2]) for c in cev)}
     if dist is not None:
-        phase_ms["allreduce"] = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
-    del percall, norm_graph, fb_graph
+        phase_ms["allreduce"] = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    del percall, step_graph, norm_marked
 
-    # ---- norm calls back to back (a throughput figure beside the in-step call): ten calls in
+    # ---- norm calls back to back (a throughput figure beside the single call): ten calls in
     # one CUDA graph, no L2 flush between them (W0, A and B exceed L2 at the workloads that
     # have a roofline), timed with events around each replay, as the burst peak is measured.
     nb_calls, nb_reps = 10, 5
@@ -623,7 +634,8 @@ def run_ours(args, wl, cfg, dist=None, extras=True):
     nk = kernels.get("norm_gemm")
     norm_roof = {"bound": "tensor", "achieved": norm_call_tflops, "peak": P_burst, "unit": "TFLOP/s",
                  "frac": norm_call_tflops / P_burst, "call_us": 1e3 * phase_ms["norm"],
-                 "flops": nf, "peak_source": f"{peak_src} (bf16_tflops, burst)"}
+                 "flops": nf, "peak_source": f"{peak_src} (bf16_tflops, burst)",
+                 "timing": f"one call after an L2 flush, event nodes inside its own graph, mean of {nprof}"}
     if nk is not None:
         norm_roof["norm_gemm_us"] = nk["us"]
         norm_roof["norm_gemm_tflops"] = nk["tflops"]
@@ -796,8 +808,9 @@ def _table(args):
     out = ["# Layer step per workload, one B200",
            "",
            f"`python bench.py --table {os.path.basename(args.table)} --steps {args.steps} --warmup {args.warmup}`: "
-           "per workload the layer step (dora_norm as one CUDA graph, dora_forward + dora_backward as a second; "
-           "the forward and backward times from one graph per call, after the timed region; "
+           "per workload the layer step (one CUDA graph of dora_norm, dora_forward and dora_backward; the per-call "
+           "times after the timed region, each call after an L2 flush: the norm by event nodes inside a graph "
+           "of that call alone, the forward and backward one graph per call; "
            "L2 flushed before every timed step, CUDA events on the launching stream), synthetic inputs of "
            "the workload's shapes. The layer roofline is the slower of flops / measured burst bf16 peak and "
            "bytes / measured HBM copy rate per call.",
@@ -828,8 +841,9 @@ def workload_config(wl, world):
     return {"workload": wl.name, "d_out": wl.d_out, "d_in": wl.d_in, "r": wl.r, "s": wl.s,
             "tokens_per_gpu": wl.T, "global_tokens": wl.T * world, "parallelism": f"dp{world}",
             "l2": "flushed before every timed step (256 MB write)",
-            "timing": "step: two CUDA graphs (norm; forward + backward) between CUDA events, max over ranks; "
-                      "call_us forward and backward: one graph per call after the timed region"}
+            "timing": "step: one CUDA graph (norm, forward, backward) between CUDA events, max over ranks; "
+                      "call_us, after the timed region, each call after an L2 flush: norm by event nodes inside "
+                      "a graph of the call alone, forward and backward one graph per call"}
 
 
 def main(argv=None):
