@@ -171,3 +171,39 @@ def test_zero_norm_row_propagates():
     keep = np.arange(wl.d_out) != 5
     assert np.max(np.abs(C[keep] - ref["C"][keep]) / ref["C"][keep]) <= tl.NORM_RTOL
     tl.check_tensor("y (other rows)", out["y"][:, torch.from_numpy(keep).cuda()], ref["y"][:, keep], "bf16")
+
+
+@pytest.mark.parametrize("key,ov", [("c4a", {}), ("c2", dict(d_out=1024, d_in=4096, T=1024)),
+                                    ("c4b", {})])
+def test_backward_fork_matches_serial(key, ov):
+    """At these sizes dx leaves SM pairs idle and runs on the library's second stream beside the
+    grouped dB/dA launch. Its results must be the serial backward's bits (the kernel profiler keeps
+    the backward serial), eagerly and replayed from a CUDA graph holding the two branches."""
+    wl = workload(key, **ov)
+    inp = tl.prepare(wl)
+    dev = tl.to_device(inp)
+    a = tl.run_gpu(dev, wl.s)
+    dw.dora_profile_start(64)
+    try:
+        b = tl.run_gpu(dev, wl.s)
+    finally:
+        dw.dora_profile_stop()
+    for k in ("dm", "dA", "dB", "dx"):
+        assert torch.equal(a[k], b[k]), k
+    W0 = dev["W0"]
+    d_out, d_in = W0.shape
+    r, T = dev["A"].shape[0], dev["x"].shape[0]
+    ws = torch.empty(max(dw.dora_workspace_size(d_out, d_in, r, W0.dtype, wl.s, T, dw.DORA_OP_BACKWARD), 256),
+                     dtype=torch.uint8, device=W0.device)
+    outs = dict(dm=tl.poisoned((d_out,), torch.float32), dA=tl.poisoned((r, d_in), W0.dtype),
+                dB=tl.poisoned((d_out, r), W0.dtype), dx=tl.poisoned((T, d_in), W0.dtype))
+    torch.cuda.synchronize()
+    gph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gph):
+        dw.dora_backward(dev["dy"], dev["x"], W0, dev["A"], dev["B"], a["C"], a["g"], a["su"], a["pre"], wl.s,
+                         ws=ws, **outs)
+    gph.replay()
+    torch.cuda.synchronize()
+    for k in ("dm", "dA", "dB", "dx"):
+        assert torch.equal(outs[k], a[k]), f"{k} (graph)"
+    del gph
