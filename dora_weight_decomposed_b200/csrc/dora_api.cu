@@ -171,26 +171,30 @@ static ClusterChoice choose_narrow_cluster_bn(int64_t M, int64_t N, int64_t K, i
   return c;
 }
 
-// The 256 x 256 base GEMMs (forward, dx): the persistent pair kernel (1) or, when
-// its tiles are too few to fill the SM pairs, clusters of 2 to 4 pairs that split
-// K. Estimated microseconds at ~1.9 GHz: a pair k-block takes the longer of its
-// MMAs and its operand loads (~110 GB/s per SM); each wave adds 1.5 us (prologue,
-// pipeline fill, last epilogue), each extra split 1.5 us of reduction, and a
-// cluster launch 1 us for its stores. The persistent kernel overlaps each tile's
-// epilogue with the next tile's main loop, so only its waves count. (256 x 128
-// cluster tiles, twice as many, measured slower: 25.2 against 22.6 us for the c4a
-// forward.)
+// The 256 x 256 base GEMMs (forward, dx): the persistent pair kernel (0) or clusters of
+// 1 to 4 pairs (the cluster kernel; with more than one pair per cluster the pairs split K).
+// Estimated microseconds at ~1.9 GHz: a pair k-block takes the longer of its MMAs and its
+// operand loads (~110 GB/s per SM); each wave adds 1.5 us (prologue, pipeline fill), each
+// extra split 1.5 us of reduction, and a cluster launch 1 us for its stores. The persistent
+// kernel overlaps each tile's epilogue with the next tile's main loop, so only its waves count,
+// except in a single wave of one tile per pair: nothing hides that epilogue's row-per-thread
+// stores (~8 us for the forward's two outputs), where the cluster kernel stores from shared
+// memory (c4b forward: 48 tiles of 33 k-blocks took 33.4 us persistent under ncu, the c4a
+// forward's 3-pair clusters with the same k-blocks per pair 23.2 us). (256 x 128 cluster
+// tiles, twice as many, measured slower: 25.2 against 22.6 us for the c4a forward.)
 static int choose_wide_cs(int64_t M, int64_t N, int64_t K, int sms) {
   const int64_t tiles = cdiv(M, 256) * cdiv(N, 256);
   const int64_t kb = std::max<int64_t>(cdiv(K, 64), 1);
   const int pairs = std::max(1, sms / 2);
   const double kb_us = std::max(2.0 * 256.0 * 256.0 * 64.0 / 23.0e6, (16384.0 + 64.0 * 256.0) / 110.0e3);
-  double best = (double)cdiv(tiles, pairs) * ((double)kb * kb_us + 1.5);
-  int cs = 1;
-  for (int c : {2, 3, 4}) {
-    if (kb < 2 * c) break;
-    const double t =
-        (double)cdiv(tiles, resident_clusters(c, sms)) * ((double)cdiv(kb, c) * kb_us + 1.5) + 1.5 * (c - 1) + 1.0;
+  const int64_t waves = cdiv(tiles, pairs);
+  double best = (double)waves * ((double)kb * kb_us + 1.5) + (waves == 1 ? 8.0 : 0.0);
+  int cs = 0;
+  for (int c : {1, 2, 3, 4}) {
+    if (c > 1 && kb < 2 * c) break;
+    const int64_t rc = resident_clusters(c, sms);
+    if (c == 1 && tiles > rc) continue;  // one pair per tile only in a single wave
+    const double t = (double)cdiv(tiles, rc) * ((double)cdiv(kb, c) * kb_us + 1.5) + 1.5 * (c - 1) + 1.0;
     if (t < best - 1e-9) {
       best = t;
       cs = c;
@@ -239,7 +243,7 @@ static void plan_backward_fork(Plan& p, int64_t d_out, int64_t d_in, int64_t r, 
   const double kb_us = std::max(2.0 * 256.0 * 256.0 * 64.0 / 23.0e6, (16384.0 + 64.0 * 256.0) / 110.0e3);
   int64_t used;
   double dx_us;
-  if (p.dx_cs == 1) {
+  if (p.dx_cs == 0) {
     const int64_t waves = cdiv(tiles, pairs);
     used = cdiv(tiles, waves);
     dx_us = (double)waves * ((double)kb * kb_us + 1.5);

@@ -1108,7 +1108,7 @@ dora_status_t bf16_forward(const dora_desc_t& d, const Plan& p, int64_t T, const
   ba.split.splits = 1;
   ba.name = "fwd_compose_gemm";
   ba.split.kb_per_split = (int)(ceil_div(d_in, kBK) + ceil_div(r, kBK));
-  if (p.fwd_cs > 1) {
+  if (p.fwd_cs >= 1) {
     // Few tiles (small token batches): clusters of pairs split K and compose in the reduction.
     const ClusterOut o{reinterpret_cast<__nv_bfloat16*>(y), reinterpret_cast<__nv_bfloat16*>(pre_save), gm1, d_out,
                        1.0f, 0, 1};
@@ -1221,7 +1221,7 @@ static dora_status_t backward_dx(const Plan& p, int Ti, int d_out, int d_in, int
     a.name = "dx_gemm";
     a.split.kb_per_split = (int)(ceil_div(d_out, kBK) + ceil_div(r, kBK));
     cudaError_t e;
-    if (p.dx_cs > 1) {
+    if (p.dx_cs >= 1) {
       const ClusterOut o{reinterpret_cast<__nv_bfloat16*>(dx), nullptr, nullptr, d_in, 1.0f, 0, 0};
       e = pair_cluster_cs<256, false, true>(p.dx_cs, a, o, st);
     } else {

@@ -26,13 +26,13 @@ struct Plan {
   int norm_bn = 0;
   size_t off_gs = 0, off_norm_part = 0;
   // forward: u = s x A^T on CTA-pair clusters (tile width, pairs per cluster = K splits);
-  // the base GEMM persistent (fwd_cs = 1) or, for few tiles, on clusters of fwd_cs pairs
-  int u_bn = 0, u_cs = 1, fwd_cs = 1;
+  // the base GEMM persistent (fwd_cs = 0) or, for few tiles, on clusters of fwd_cs pairs
+  int u_bn = 0, u_cs = 1, fwd_cs = 0;
   size_t off_su = 0;
   // backward: du, dB, dA on pair clusters; dx like the base GEMM
   int dm_rowblocks = 0, dm_rows = 256;
   // (dB_grouped: dB and dA in one grouped launch of whole tiles, both dB_bn wide)
-  int du_bn = 0, du_cs = 1, dB_bn = 0, dB_cs = 1, dA_bn = 0, dA_cs = 1, dx_cs = 1, dBA_grouped = 0;
+  int du_bn = 0, du_cs = 1, dB_bn = 0, dB_cs = 1, dA_bn = 0, dA_cs = 1, dx_cs = 0, dBA_grouped = 0;
   // dx and the grouped dB/dA launch both follow du alone; when dx's tiles leave SM pairs
   // free (bwd_fork), dx runs on a second stream on dx_pairs pairs, dB/dA beside it on dBA_pairs
   int bwd_fork = 0, dx_pairs = 0, dBA_pairs = 0;
