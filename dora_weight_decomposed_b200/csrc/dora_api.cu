@@ -338,6 +338,22 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
       p.u_bn = u.bn;
       p.u_cs = u.cs;
       p.fwd_cs = choose_wide_cs(T, d_out, cdiv(d_in, 64) * 64 + cdiv(r, 64) * 64, p.sms);
+      // The base GEMM needs s u only for its last k-block: when its CTAs and u's fit on the
+      // SMs together (one wave each), it starts its x W0 main loop beside u.
+      {
+        const int64_t tiles_u = cdiv(T, 256) * cdiv(r, p.u_bn);
+        const int64_t tiles_f = cdiv(T, 256) * cdiv(d_out, 256);
+        const int64_t ctas_u = 2 * p.u_cs * tiles_u;
+        bool one_wave = tiles_u <= resident_clusters(p.u_cs, p.sms);
+        int64_t ctas_f;
+        if (p.fwd_cs >= 1) {
+          ctas_f = 2 * p.fwd_cs * tiles_f;
+          one_wave = one_wave && tiles_f <= resident_clusters(p.fwd_cs, p.sms);
+        } else {
+          ctas_f = 2 * std::min<int64_t>(tiles_f, std::max(1, p.sms / 2));
+        }
+        p.fwd_defer = (one_wave && ctas_u + ctas_f <= p.sms) ? 1 : 0;
+      }
       p.off_su = take((size_t)T * r * 2);
     } else if ((op == DORA_OP_BACKWARD || op == DORA_OP_BACKWARD_FULL) && T > 0) {
       p.off_dz = take((size_t)T * d_out * 2);

@@ -140,7 +140,8 @@ struct GemmArgs {
   int M = 0, N = 0;
   Split split;
   int a1_kwrap = 0;  // see GemmGeom::a1_kwrap
-  int defer_wait_src1 = 0;  // see GemmGeom::defer_wait_src1 (CTA-pair split kernel)
+  int defer_wait_src1 = 0;  // see GemmGeom::defer_wait_src1 (CTA-pair kernels)
+  int wait_then_trigger = 0;  // see GemmGeom::wait_then_trigger
   const char* name = "gemm";
 };
 
@@ -215,7 +216,7 @@ static cudaError_t launch_gemm_pair(const GemmArgs& g, const typename Epi::Param
     tb1 = tb0;
   }
   const int kps = g.split.kb_per_split > 0 ? g.split.kb_per_split : kb0 + kb1;
-  GemmGeom geom{g.M, g.N, kb0, kb1, kps, g.a1_kwrap};
+  GemmGeom geom{g.M, g.N, kb0, kb1, kps, g.a1_kwrap, g.defer_wait_src1, g.wait_then_trigger};
   const long long splits = ceil_div(std::max(kb0 + kb1, 1), kps);
   const long long items = ceil_div(g.N, Cfg::BN) * ceil_div(g.M, 2 * kBM) * splits;
   const long long pairs = std::max<long long>(1, std::min<long long>(items, sms / 2));
@@ -741,7 +742,7 @@ static cudaError_t launch_pair_cluster(const GemmArgs& g, const ClusterOut& o, c
     tb1 = tb0;
   }
   const int kb = std::max(kb0 + kb1, 1);
-  GemmGeom geom{g.M, g.N, kb0, kb1, (int)ceil_div(kb, CS), 0, 0};
+  GemmGeom geom{g.M, g.N, kb0, kb1, (int)ceil_div(kb, CS), 0, g.defer_wait_src1, g.wait_then_trigger};
   const long long tiles = ceil_div(g.N, Cfg::BN) * ceil_div(g.M, 2 * kBM);
   auto kern = gemm_sm100_pair_cluster_kernel<Cfg, CS>;
   constexpr int smem_bytes = PairClusterLayout<Cfg>::SMEM_BYTES;
@@ -1092,6 +1093,9 @@ dora_status_t bf16_forward(const dora_desc_t& d, const Plan& p, int64_t T, const
   ua.M = Ti;
   ua.N = r;
   ua.name = "u_gemm";
+  // Under fwd_defer the base GEMM below starts its x W0 main loop beside this one and waits
+  // for it only before loading su: this grid then waits for its own predecessor first.
+  ua.wait_then_trigger = p.fwd_defer;
   cudaError_t e = narrow_cluster<false, false>(p.u_bn, p.u_cs, ua, d.s, su, r, false, st);
   if (e != cudaSuccess) return gemm_status(e, "dora_forward: LoRA down projection");
 
@@ -1107,6 +1111,7 @@ dora_status_t bf16_forward(const dora_desc_t& d, const Plan& p, int64_t T, const
   ba.N = d_out;
   ba.split.splits = 1;
   ba.name = "fwd_compose_gemm";
+  ba.defer_wait_src1 = p.fwd_defer;
   ba.split.kb_per_split = (int)(ceil_div(d_in, kBK) + ceil_div(r, kBK));
   if (p.fwd_cs >= 1) {
     // Few tiles (small token batches): clusters of pairs split K and compose in the reduction.

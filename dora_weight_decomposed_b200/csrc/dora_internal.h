@@ -28,6 +28,9 @@ struct Plan {
   // forward: u = s x A^T on CTA-pair clusters (tile width, pairs per cluster = K splits);
   // the base GEMM persistent (fwd_cs = 0) or, for few tiles, on clusters of fwd_cs pairs
   int u_bn = 0, u_cs = 1, fwd_cs = 0;
+  // the base GEMM launched beside u (both fit on the SMs at once): it waits for u only
+  // before its su k-block
+  int fwd_defer = 0;
   size_t off_su = 0;
   // backward: du, dB, dA on pair clusters; dx like the base GEMM
   int dm_rowblocks = 0, dm_rows = 256;

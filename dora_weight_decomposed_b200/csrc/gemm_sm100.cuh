@@ -37,12 +37,29 @@ struct GemmGeom {
   int kb1;           // k-blocks taken from source 1
   int kb_per_split;  // k-blocks per blockIdx.z
   int a1_kwrap;      // > 0: source-1 A coordinates wrap modulo this many K elements
-  // CTA-pair split kernel only: nonzero when only the source-1 operands come from
-  // the preceding grid. The kernel then starts its source-0 main loop at once;
-  // the producer waits for the preceding grid just before its first source-1
-  // load, and the epilogue warps before they write anything.
+  // CTA-pair kernels (persistent, split, cluster): nonzero when only the source-1
+  // operands come from the preceding grid. The kernel then starts its source-0
+  // main loop at once; the producer waits for the preceding grid just before its
+  // first source-1 load, and the epilogue (or the cluster reduction) before it
+  // writes anything. Only valid after a grid that waits for its own predecessor
+  // before it triggers (wait_then_trigger, or the Gram kernel), so that all work
+  // before that grid is complete when this one starts.
   int defer_wait_src1 = 0;
+  // Persistent and cluster kernels: wait for the preceding grid before letting
+  // the dependent grid launch (see defer_wait_src1).
+  int wait_then_trigger = 0;
 };
+
+// The dependent-launch handshake at the end of a CTA-pair kernel's prologue.
+__device__ __forceinline__ void pdl_handshake(const GemmGeom& geom) {
+  if (geom.wait_then_trigger) {
+    pdl_wait();
+    pdl_trigger();
+  } else {
+    pdl_trigger();
+    if (!geom.defer_wait_src1) pdl_wait();
+  }
+}
 
 template <int BN_, bool A_MN_, bool B_MN_>
 struct GemmCfg {
@@ -470,13 +487,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  pdl_trigger();
-  pdl_wait();
+  pdl_handshake(geom);
+  const bool defer = geom.defer_wait_src1 != 0 && !geom.wait_then_trigger;
 
   if (warp == 0) {
     if (lane == 0) {
       int it = 0;
       bool ok = true;
+      bool waited = !defer;
 #pragma unroll 1
       for (int item = pair; item < items && ok; item += npairs) {
         const int t = item / splits, split = item - t * splits;
@@ -497,8 +515,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           uint8_t* sa = smem + s * Cfg::STAGE_BYTES;
           uint8_t* sb = sa + Cfg::A_BYTES;
           const uint32_t fb = mapa_shared(smem_u32(&full[s]), 0);
-          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
           const bool src1 = kb >= geom.kb0;
+          if (src1 && !waited) {
+            pdl_wait();  // the source-1 operands come from the preceding grid
+            waited = true;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
           const int k0 = (src1 ? kb - geom.kb0 : kb) * kBK;
           const int k0a = (src1 && geom.a1_kwrap > 0) ? k0 % geom.a1_kwrap : k0;
           const CUtensorMap* ta = src1 ? &tA1 : &tA0;
@@ -578,6 +600,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;
     const int row = q * 32 + lane;
     typename Epi::RowState st{};
+    if (defer) pdl_wait();  // before the epilogue reads or writes anything
     int j = 0;
 #pragma unroll 1
     for (int item = pair; item < items; item += npairs, ++j) {
@@ -953,13 +976,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  pdl_trigger();
-  pdl_wait();
+  pdl_handshake(geom);
+  const bool defer = geom.defer_wait_src1 != 0 && !geom.wait_then_trigger;
 
   if (warp == 0) {
     if (lane == 0) {
       const int nb0 = tn * Cfg::BN + (int)q * Cfg::H0;
       const int nb1 = tn * Cfg::BN + Cfg::N0 + (int)q * Cfg::H1;
+      bool waited = !defer;
 #pragma unroll 1
       for (int i = 0; i < nkb; ++i) {
         const int s = i % STAGES;
@@ -967,9 +991,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint8_t* sa = smem + s * Cfg::STAGE_BYTES;
         uint8_t* sb = sa + Cfg::A_BYTES;
         const uint32_t fb = mapa_shared(smem_u32(&full[s]), leader);
-        if (q == 0) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
         const int kb = kb_begin + i;
         const bool src1 = kb >= geom.kb0;
+        if (src1 && !waited) {
+          pdl_wait();  // the source-1 operands come from the preceding grid
+          waited = true;
+        }
+        if (q == 0) mbar_arrive_expect_tx(&full[s], 2 * Cfg::STAGE_BYTES);
         const int k0 = (src1 ? kb - geom.kb0 : kb) * kBK;
         const CUtensorMap* ta = src1 ? &tA1 : &tA0;
         const CUtensorMap* tb = src1 ? &tB1 : &tB0;
@@ -1030,6 +1058,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 
   // ---- reduction inside the cluster, CW columns per round
+  if (defer) pdl_wait();  // before the reduction reads or writes anything global
   bool acc_ok = true;
   if (warp >= 2) {
     // tcgen05.ld is warp-collective: the whole warp takes the same branch below.
