@@ -233,6 +233,7 @@ static bool dBA_grouped(int64_t d_out, int64_t d_in, int64_t r, int64_t T, int b
 static void plan_backward_fork(Plan& p, int64_t d_out, int64_t d_in, int64_t r, int64_t T) {
   const int pairs = std::max(1, p.sms / 2);
   p.bwd_fork = 0;
+  p.dx_defer = 0;
   p.dx_pairs = pairs;
   p.dBA_pairs = pairs;
   if (!p.dBA_grouped) return;
@@ -263,6 +264,15 @@ static void plan_backward_fork(Plan& p, int64_t d_out, int64_t d_in, int64_t r, 
   p.bwd_fork = 1;
   p.dx_pairs = (int)used;
   p.dBA_pairs = (int)std::min(idle, tBA);
+  // dx needs du only for its last k-block ([dz | du] [W0 ; A]): when du's CTAs and dx's fit
+  // on the SMs together (one wave each), dx starts beside du, and dB/dA follow their own copy
+  // of du on the second stream. That stream then carries du and all of dB/dA, so only where
+  // dB/dA take at most two tiles per pair (measured: c4a backward 38.9 -> 32.9 us, c4b
+  // 51.2 -> 45.1 us; c3 at T = 256, seven tiles per pair, 141.4 -> 145.5 us).
+  const int64_t tiles_du = cdiv(T, 256) * cdiv(r, p.du_bn);
+  if (tiles_du <= resident_clusters(p.du_cs, p.sms) && 2 * p.du_cs * tiles_du + 2 * used <= p.sms &&
+      cdiv(tBA, p.dBA_pairs) <= 2)
+    p.dx_defer = 1;
 }
 
 static NarrowChoice choose_narrow(int64_t M, int64_t N, int64_t K, bool b_mn, int sms) {
@@ -370,6 +380,7 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
       p.du_bn = du.bn;
       p.du_cs = du.cs;
       p.off_du = take((size_t)T * r * 2);
+      p.off_du2 = take((size_t)T * r * 2);  // always, so that the workspace grows with T
       const ClusterChoice dB = choose_narrow_cluster(d_out, r, T, true, p.sms);
       p.dB_bn = dB.bn;
       p.dB_cs = dB.cs;

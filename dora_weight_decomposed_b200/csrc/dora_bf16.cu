@@ -89,8 +89,8 @@ static bool make_map(CUtensorMap* map, const Mat& m, int box_outer, const char* 
 // Launch with programmatic stream serialization so the kernel's prologue can
 // overlap the previous kernel's tail (see pdl_wait / pdl_trigger).
 template <class... KArgs, class... Args>
-static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                              Args&&... args) {
+static cudaError_t launch_pdl_if(bool early, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t st, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -99,10 +99,16 @@ static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   // Under the kernel profiler each launch is timed on its own: no early start.
-  attr[0].val.programmaticStreamSerializationAllowed = profiling_on() ? 0 : 1;
+  attr[0].val.programmaticStreamSerializationAllowed = (early && !profiling_on()) ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+template <class... KArgs, class... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  return launch_pdl_if(true, kern, grid, block, smem, st, std::forward<Args>(args)...);
 }
 
 static dora_status_t gemm_status(cudaError_t e, const char* where) {
@@ -895,7 +901,7 @@ static cudaError_t narrow_cluster(int bn, int cs, const GemmArgs& g, float alpha
 // launch (gemm_sm100_pair_grouped_kernel): whole tiles, at most `pairs` CTA pairs.
 template <class Cfg>
 static cudaError_t launch_grouped(const GemmArgs* gs, const ClusterOut* os, int nprob, int pairs, const char* name,
-                                  cudaStream_t st) {
+                                  cudaStream_t st, bool early = true) {
   GroupMaps maps{};
   GroupGeom geom{};
   const int a_box = Cfg::A_MN ? 64 : kBM;
@@ -950,7 +956,7 @@ static cudaError_t launch_grouped(const GemmArgs* gs, const ClusterOut* os, int 
   }
   {
     ProfRange pr(name, st);
-    e = launch_pdl(kern, dim3((unsigned)(2 * P)), dim3(kGemmThreads), (size_t)smem_bytes, st, maps, geom);
+    e = launch_pdl_if(early, kern, dim3((unsigned)(2 * P)), dim3(kGemmThreads), (size_t)smem_bytes, st, maps, geom);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) t_detail = "grouped launch, " + std::to_string(tiles) + " tiles on " + std::to_string(P) + " pairs";
@@ -959,14 +965,14 @@ static cudaError_t launch_grouped(const GemmArgs* gs, const ClusterOut* os, int 
 
 template <bool A_MN, bool B_MN>
 static cudaError_t grouped_bn(int bn, const GemmArgs* gs, const ClusterOut* os, int nprob, int pairs,
-                              const char* name, cudaStream_t st) {
+                              const char* name, cudaStream_t st, bool early = true) {
   if constexpr (!B_MN) {
-    if (bn == 64) return launch_grouped<PairCfg<64, A_MN, B_MN>>(gs, os, nprob, pairs, name, st);
+    if (bn == 64) return launch_grouped<PairCfg<64, A_MN, B_MN>>(gs, os, nprob, pairs, name, st, early);
   }
-  if (bn == 128) return launch_grouped<PairCfg<128, A_MN, B_MN>>(gs, os, nprob, pairs, name, st);
-  if (bn == 256) return launch_grouped<PairCfg<256, A_MN, B_MN>>(gs, os, nprob, pairs, name, st);
-  if (bn == 384) return launch_grouped<PairCfg<384, A_MN, B_MN>>(gs, os, nprob, pairs, name, st);
-  if (bn == 512) return launch_grouped<PairCfg<512, A_MN, B_MN>>(gs, os, nprob, pairs, name, st);
+  if (bn == 128) return launch_grouped<PairCfg<128, A_MN, B_MN>>(gs, os, nprob, pairs, name, st, early);
+  if (bn == 256) return launch_grouped<PairCfg<256, A_MN, B_MN>>(gs, os, nprob, pairs, name, st, early);
+  if (bn == 384) return launch_grouped<PairCfg<384, A_MN, B_MN>>(gs, os, nprob, pairs, name, st, early);
+  if (bn == 512) return launch_grouped<PairCfg<512, A_MN, B_MN>>(gs, os, nprob, pairs, name, st, early);
   t_detail = "no grouped tile of width " + std::to_string(bn);
   return cudaErrorInvalidValue;
 }
@@ -1159,7 +1165,7 @@ dora_status_t bf16_merge(const dora_desc_t& d, const Plan& p, const void* W0, co
 // cluster split-K launches when their tiles are too few for the SM pairs.
 static dora_status_t backward_dBA(const Plan& p, int Ti, int d_out, int d_in, int r, const __nv_bfloat16* dz,
                                   const void* su, const void* x, const __nv_bfloat16* du, void* dA, void* dB,
-                                  int pairs, cudaStream_t st) {
+                                  int pairs, cudaStream_t st, bool early = true) {
   if (p.dBA_grouped) {
     GemmArgs a[2];
     a[0].a0 = Mat{dz, Ti, d_out, d_out};
@@ -1174,7 +1180,7 @@ static dora_status_t backward_dBA(const Plan& p, int Ti, int d_out, int d_in, in
     a[1].N = r;
     const ClusterOut o[2] = {{reinterpret_cast<__nv_bfloat16*>(dB), nullptr, nullptr, r, 1.0f, 0, 0},
                              {reinterpret_cast<__nv_bfloat16*>(dA), nullptr, nullptr, d_in, 1.0f, 1, 0}};
-    cudaError_t e = grouped_bn<true, true>(p.dB_bn, a, o, 2, pairs, "dBA_gemm", st);
+    cudaError_t e = grouped_bn<true, true>(p.dB_bn, a, o, 2, pairs, "dBA_gemm", st, early);
     if (e != cudaSuccess) return gemm_status(e, "dora_backward: dB and dA");
   } else {
     // dB = dz^T su  (both token-major: K = T)
@@ -1208,10 +1214,11 @@ static dora_status_t backward_dBA(const Plan& p, int Ti, int d_out, int d_in, in
 }
 
 // dx = [dz | du] [W0 ; A]  (W0 and A read MN-major: K rows, N = d_in contiguous); the
-// persistent kernel on at most sms / 2 pairs.
+// persistent kernel on at most sms / 2 pairs; with defer, dx directly follows the du launch
+// and waits for it only before its du k-block (du having waited for its own predecessor).
 static dora_status_t backward_dx(const Plan& p, int Ti, int d_out, int d_in, int r, const __nv_bfloat16* dz,
                                  const __nv_bfloat16* du, const void* W0, const void* A, void* dx, int sms,
-                                 cudaStream_t st) {
+                                 bool defer, cudaStream_t st) {
   {
     GemmArgs a;
     a.a0 = Mat{dz, Ti, d_out, d_out};
@@ -1224,6 +1231,7 @@ static dora_status_t backward_dx(const Plan& p, int Ti, int d_out, int d_in, int
     a.N = d_in;
     a.split.splits = 1;
     a.name = "dx_gemm";
+    a.defer_wait_src1 = defer ? 1 : 0;
     a.split.kb_per_split = (int)(ceil_div(d_out, kBK) + ceil_div(r, kBK));
     cudaError_t e;
     if (p.dx_cs >= 1) {
@@ -1310,8 +1318,8 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
       if (e != cudaSuccess) return cuda_status(e, "dora_backward: compose backward");
     }
   }
-  // du = s dz B  (B read MN-major: K = d_out rows, N = r contiguous)
-  {
+  // du = s dz B  (B read MN-major: K = d_out rows, N = r contiguous), into `out` on `ss`
+  auto launch_du = [&](__nv_bfloat16* out, bool wait_then_trigger, cudaStream_t ss) {
     GemmArgs a;
     a.a0 = Mat{dz, Ti, d_out, d_out};
     a.b0 = Mat{B, d_out, r, r};
@@ -1319,30 +1327,64 @@ dora_status_t bf16_backward(const dora_desc_t& d, const Plan& p, int64_t T, cons
     a.M = Ti;
     a.N = r;
     a.name = "du_gemm";
-    cudaError_t e = narrow_cluster<false, true>(p.du_bn, p.du_cs, a, d.s, du, r, false, st);
-    if (e != cudaSuccess) return gemm_status(e, "dora_backward: du");
-  }
-  // dx and dB/dA both follow du and nothing else. Under the plan's fork dx goes to the
-  // second stream, on the pairs its tiles need, and the grouped dB/dA launch takes the
-  // idle pairs beside it; the caller's stream waits for both before this call returns.
-  // (Serial when the kernel profiler times each launch on its own.)
+    a.wait_then_trigger = wait_then_trigger ? 1 : 0;
+    return gemm_status(narrow_cluster<false, true>(p.du_bn, p.du_cs, a, d.s, out, r, false, ss), "dora_backward: du");
+  };
+  auto fork = [&](SideStream* ss) {
+    cudaError_t e = cudaEventRecord(ss->fork, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->s, ss->fork, 0);
+    return cuda_status(e, "dora_backward: forking onto the second stream");
+  };
+  auto join = [&](SideStream* ss) {
+    cudaError_t e = cudaEventRecord(ss->join, ss->s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ss->join, 0);
+    return cuda_status(e, "dora_backward: joining the second stream");
+  };
+  // dx and dB/dA both follow du and nothing else. Under the plan's fork dx and the grouped
+  // dB/dA launch run at once, on two streams, each on its own share of the SM pairs; the
+  // caller's stream waits for both before this call returns. (Serial when the kernel
+  // profiler times each launch on its own.)
   SideStream* side = (p.bwd_fork && dx && !profiling_on()) ? side_stream(st) : nullptr;
+  if (side && p.dx_defer) {
+    // dx also starts beside du: du, then dx on the caller's stream with nothing between
+    // them (du waits for compose before letting dx launch; dx waits for du only before its
+    // du k-block). dB/dA, forked right after compose, take their own copy of du from the
+    // same kernel (the same bits) on the second stream, so that no event sits between du
+    // and dx.
+    __nv_bfloat16* du2 = reinterpret_cast<__nv_bfloat16*>(ws + p.off_du2);
+    dora_status_t status = fork(side);
+    if (status != DORA_OK) return status;
+    status = launch_du(du2, false, side->s);
+    // (dB/dA launch only once their du copy is complete: launched early they would hold
+    // their pairs while du runs, and dx could not start all its tiles beside du.)
+    const dora_status_t dBA_status =
+        status != DORA_OK ? status
+                          : backward_dBA(p, Ti, d_out, d_in, r, dz, su, x, du2, dA, dB, p.dBA_pairs, side->s, false);
+    status = launch_du(du, true, st);
+    const dora_status_t dx_status =
+        status != DORA_OK ? status : backward_dx(p, Ti, d_out, d_in, r, dz, du, W0, A, dx, 2 * p.dx_pairs, true, st);
+    status = join(side);
+    if (status != DORA_OK) return status;
+    return dBA_status != DORA_OK ? dBA_status : dx_status;
+  }
+  {
+    const dora_status_t status = launch_du(du, false, st);
+    if (status != DORA_OK) return status;
+  }
   if (!side) {
     const dora_status_t status = backward_dBA(p, Ti, d_out, d_in, r, dz, su, x, du, dA, dB, p.sms / 2, st);
     if (status != DORA_OK || !dx) return status;
-    return backward_dx(p, Ti, d_out, d_in, r, dz, du, W0, A, dx, p.sms, st);
+    return backward_dx(p, Ti, d_out, d_in, r, dz, du, W0, A, dx, p.sms, false, st);
   }
   {
-    cudaError_t e = cudaEventRecord(side->fork, st);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s, side->fork, 0);
-    if (e != cudaSuccess) return cuda_status(e, "dora_backward: forking dx onto the second stream");
+    const dora_status_t status = fork(side);
+    if (status != DORA_OK) return status;
   }
   const dora_status_t dBA_status = backward_dBA(p, Ti, d_out, d_in, r, dz, su, x, du, dA, dB, p.dBA_pairs, st);
-  const dora_status_t dx_status = backward_dx(p, Ti, d_out, d_in, r, dz, du, W0, A, dx, 2 * p.dx_pairs, side->s);
+  const dora_status_t dx_status = backward_dx(p, Ti, d_out, d_in, r, dz, du, W0, A, dx, 2 * p.dx_pairs, false, side->s);
   {
-    cudaError_t e = cudaEventRecord(side->join, side->s);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, side->join, 0);
-    if (e != cudaSuccess) return cuda_status(e, "dora_backward: joining the second stream");
+    const dora_status_t status = join(side);
+    if (status != DORA_OK) return status;
   }
   return dBA_status != DORA_OK ? dBA_status : dx_status;
 }

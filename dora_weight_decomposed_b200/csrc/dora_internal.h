@@ -39,7 +39,10 @@ struct Plan {
   // dx and the grouped dB/dA launch both follow du alone; when dx's tiles leave SM pairs
   // free (bwd_fork), dx runs on a second stream on dx_pairs pairs, dB/dA beside it on dBA_pairs
   int bwd_fork = 0, dx_pairs = 0, dBA_pairs = 0;
-  size_t off_dz = 0, off_dm_part = 0, off_du = 0;
+  // under the fork, dx also starts beside du when both fit on the SMs at once (dx_defer);
+  // dB/dA then take a second copy of du (off_du2), computed on their own stream
+  int dx_defer = 0;
+  size_t off_dz = 0, off_dm_part = 0, off_du = 0, off_du2 = 0;
   // full (non-detached) gradient: kappa, kappa-scaled B, Gram, Q = W' A^T, H = s B^T diag(kappa) B
   Split q, h;
   int q_bn = 0, h_bn = 0;
