@@ -382,6 +382,26 @@ def run_reference(args, wl, cfg):
 
 # ---------------------------------------------------------------- our arm
 
+def graph_kernel_nodes(gph):
+    """Kernel nodes of a CUDA graph captured with keep_graph=True (the library's launches; its
+    memsets are memset nodes), or None when the CUDA Python bindings cannot read the graph."""
+    try:
+        from cuda.bindings import runtime as rt
+        g = rt.cudaGraph_t(init_value=int(gph.raw_cuda_graph()))
+        err, _, n = rt.cudaGraphGetNodes(g, 0)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        err, nodes, n = rt.cudaGraphGetNodes(g, n)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        kinds = [rt.cudaGraphNodeGetType(nd) for nd in nodes[:n]]
+        if any(k[0] != rt.cudaError_t.cudaSuccess for k in kinds):
+            return None
+        return sum(1 for k in kinds if k[1] == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
+    except Exception:
+        return None
+
+
 def graph_time_ms(torch, fn, flush, warmup, calls):
     """Median device time of one call of fn: a CUDA graph of the call between two event record
     nodes (events made with external=True, so that the graph's own launch is left out), replayed
@@ -468,8 +488,8 @@ def run_ours(args, wl, cfg, dist=None, extras=True):
     # ~3 us). The whole step also runs under the library's kernel profiler (each kernel launched and
     # timed on its own). (Event nodes inside the step's own graph would time the norm there too, but
     # each cost the step ~3 us: 98.0 against 95.2 us at c4a.)
-    def capture(fns, profiled=False, marks=None):
-        gph = torch.cuda.CUDAGraph()
+    def capture(fns, profiled=False, marks=None, keep=False):
+        gph = torch.cuda.CUDAGraph(keep_graph=True) if keep else torch.cuda.CUDAGraph()
         if profiled:
             dw.dora_profile_start(256)
         with torch.cuda.graph(gph):
@@ -481,15 +501,19 @@ def run_ours(args, wl, cfg, dist=None, extras=True):
                 marks[1].record()
         if profiled:
             dw.dora_profile_stop()
+        if keep:
+            gph.instantiate()
         torch.cuda.synchronize()
         return gph
 
-    step_graph = capture(calls)
+    step_graph = capture(calls, keep=True)
     norm_marks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
     norm_marked = capture([call_norm], marks=norm_marks)
     percall = [capture([c]) for c in (call_fwd, call_bwd)]
     prof = capture(calls, profiled=True)
-    launches_per_step = dw.dora_profile_count()
+    # Kernels per step: the step graph's kernel nodes (the profiled capture runs the backward
+    # serially, one du launch fewer where the backward forks); the profiler's count otherwise.
+    launches_per_step = graph_kernel_nodes(step_graph) or dw.dora_profile_count()
 
     # ---- warm-up
     for _ in range(args.warmup):
