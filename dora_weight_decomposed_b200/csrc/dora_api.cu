@@ -311,6 +311,7 @@ static NarrowChoice choose_narrow(int64_t M, int64_t N, int64_t K, bool b_mn, in
 Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
   Plan p;
   p.sms = device_sm_count();
+  p.fwd_pairs = std::max(1, p.sms / 2);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -363,6 +364,29 @@ Plan make_plan(const dora_desc_t& d, int64_t T, int op) {
           ctas_f = 2 * std::min<int64_t>(tiles_f, std::max(1, p.sms / 2));
         }
         p.fwd_defer = (one_wave && ctas_u + ctas_f <= p.sms) ? 1 : 0;
+        // A persistent base GEMM of several waves whose last wave leaves pairs idle runs the
+        // same waves on fewer pairs (ceil(tiles / waves)); u then takes the SMs left over, on
+        // the largest clusters that fit there, when it is estimated to end before the base
+        // GEMM's first tile reaches its s u k-block (c2: 128 tiles in two waves on 64 pairs,
+        // u's 8 tiles on 20 SMs).
+        const int pairs = std::max(1, p.sms / 2);
+        const int64_t waves = cdiv(tiles_f, pairs);
+        if (!p.fwd_defer && p.fwd_cs == 0 && waves >= 2) {
+          const int64_t fpairs = cdiv(tiles_f, waves);
+          const int64_t spare = p.sms - 2 * fpairs;
+          const int64_t kb_u = std::max<int64_t>(cdiv(d_in, 64), 1);
+          const int64_t kb_f = cdiv(d_in, 64) + cdiv(r, 64);
+          const double kbu_us = std::max(2.0 * 256.0 * p.u_bn * 64.0 / 23.0e6, (16384.0 + 64.0 * p.u_bn) / 110.0e3);
+          const double kbf_us = std::max(2.0 * 256.0 * 256.0 * 64.0 / 23.0e6, (16384.0 + 64.0 * 256.0) / 110.0e3);
+          int cs = 0;
+          for (int c : {1, 2, 3, 4})
+            if (2 * c * tiles_u <= spare && (c == 1 || kb_u >= 2 * c) && tiles_u <= resident_clusters(c, p.sms)) cs = c;
+          if (cs > 0 && (double)cdiv(kb_u, cs) * kbu_us + 3.0 <= (double)kb_f * kbf_us) {
+            p.u_cs = cs;
+            p.fwd_pairs = (int)fpairs;
+            p.fwd_defer = 1;
+          }
+        }
       }
       p.off_su = take((size_t)T * r * 2);
     } else if ((op == DORA_OP_BACKWARD || op == DORA_OP_BACKWARD_FULL) && T > 0) {

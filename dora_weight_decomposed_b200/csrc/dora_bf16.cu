@@ -1128,7 +1128,7 @@ dora_status_t bf16_forward(const dora_desc_t& d, const Plan& p, int64_t T, const
   }
   EpiCompose::Params cp{reinterpret_cast<__nv_bfloat16*>(y), reinterpret_cast<__nv_bfloat16*>(pre_save), gm1,
                         d_out};
-  e = launch_gemm_pair<PairCfg<256, false, false>, EpiCompose>(ba, cp, p.sms, st);
+  e = launch_gemm_pair<PairCfg<256, false, false>, EpiCompose>(ba, cp, 2 * p.fwd_pairs, st);
   return gemm_status(e, "dora_forward: base GEMM with compose");
 }
 

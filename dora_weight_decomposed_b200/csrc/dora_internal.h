@@ -31,6 +31,8 @@ struct Plan {
   // the base GEMM launched beside u (both fit on the SMs at once): it waits for u only
   // before its su k-block
   int fwd_defer = 0;
+  // pairs the persistent base GEMM runs on (fewer than the device's when u runs beside it)
+  int fwd_pairs = 74;
   size_t off_su = 0;
   // backward: du, dB, dA on pair clusters; dx like the base GEMM
   int dm_rowblocks = 0, dm_rows = 256;
