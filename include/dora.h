@@ -160,6 +160,14 @@ DORA_API dora_status_t dora_forward(const dora_desc_t* desc, int64_t T, const vo
  *      fp32 from dora_norm; su_save and pre_save from dora_forward (required).
  * Out: dm [d_out] fp32; dA [r x d_in], dB [d_out x r] (dtype);
  *      dx [T x d_in] (dtype) or NULL to skip the input gradient.
+ * Streams: for small token batches the call may run dB and dA (or dx) on a
+ * second stream owned by the library (one per host thread and device, created
+ * on the first such call outside a stream capture and kept for the life of the
+ * thread), forked from `stream` by an event after the compose backward and
+ * joined back into `stream` by an event before the call returns: work queued
+ * on `stream` afterwards sees all outputs, and a CUDA graph captured around the
+ * call holds both branches. Under the kernel profiler the call stays on
+ * `stream` alone.
  */
 DORA_API dora_status_t dora_backward(const dora_desc_t* desc, int64_t T, const void* dy, const void* x, const void* W0,
                             const void* A, const void* B, const float* norm, const float* g, const void* su_save,
