@@ -39,7 +39,8 @@ struct Plan {
   // (dB_grouped: dB and dA in one grouped launch of whole tiles, both dB_bn wide)
   int du_bn = 0, du_cs = 1, dB_bn = 0, dB_cs = 1, dA_bn = 0, dA_cs = 1, dx_cs = 0, dBA_grouped = 0;
   // dx and the grouped dB/dA launch both follow du alone; when dx's tiles leave SM pairs
-  // free (bwd_fork), dx runs on a second stream on dx_pairs pairs, dB/dA beside it on dBA_pairs
+  // free (bwd_fork), the two run at once on two streams, dx on dx_pairs pairs and dB/dA on
+  // dBA_pairs (dx on the second stream, or, with dx_defer, dB/dA there)
   int bwd_fork = 0, dx_pairs = 0, dBA_pairs = 0;
   // under the fork, dx also starts beside du when both fit on the SMs at once (dx_defer);
   // dB/dA then take a second copy of du (off_du2), computed on their own stream
